@@ -1,0 +1,353 @@
+"""Pins of the fp64 oracle against values and properties fixed elsewhere.
+
+Every pin here comes from outside the oracle: numbers the pages print
+(fixtures in tests/golden, each citing its page and section), closed forms
+from trigonometry and exponentials, invariants of rotations and of softmax,
+and brute force in plain Python loops on tiny inputs.  Each is chosen so that
+a plausible slip in the oracle (a dropped term, a wrong sign, a swapped index,
+a transposed operand, a wrong frequency exponent) fails at least one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import nomas_oracle as O
+
+COS1 = 0.5403023058681398   # cos(1 rad)
+SIN1 = 0.8414709848078965   # sin(1 rad)
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- bf16 -----
+def test_bf16_widening_exact_values():
+    # 0x3F80 = 1.0, 0xC000 = -2.0, 0x3E20 = 0.15625, 0x7F80 = +inf, 0x0001 =
+    # smallest subnormal 2^-133.
+    bits = np.array([0x3F80, 0xC000, 0x3E20, 0x7F80, 0x0001, 0x8000], dtype=np.uint16)
+    got = O.bf16_bits_to_f64(bits)
+    assert got[0] == 1.0 and got[1] == -2.0 and got[2] == 0.15625
+    assert np.isinf(got[3]) and got[3] > 0
+    assert got[4] == 2.0 ** -133
+    assert got[5] == 0.0 and math.copysign(1, got[5]) < 0
+
+
+# ------------------------------------------------------------ positions ----
+def test_video_positions_match_hand_table(golden_dir):
+    rows = np.loadtxt(os.path.join(golden_dir, "video_positions_2x2x3.txt"), dtype=np.int64)
+    t, h, w = O.video_positions(frames=2, grid_h=2, grid_w=3, t0=5)
+    assert np.array_equal(rows[:, 1], t)
+    assert np.array_equal(rows[:, 2], h)
+    assert np.array_equal(rows[:, 3], w)
+
+
+def test_token_grid_sizes_from_pages(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "cache_sizes.json")))
+    gh, gw = g["grid_720p"]
+    t, h, w = O.video_positions(g["latent_frames_per_segment"], gh, gw, 0)
+    assert gh * gw == g["tokens_per_frame_720p"]
+    assert t.size == g["tokens_per_segment"]
+    assert h.max() == gh - 1 and w.max() == gw - 1 and t.max() == 29
+
+
+# ----------------------------------------------------------------- RoPE ----
+def _one_token(vec, pos, split, theta):
+    """Rotate a single video token holding ``vec`` in every head."""
+    x = np.tile(np.asarray(vec, dtype=np.float64), (1, 2, 1))  # [1][2][D]
+    t, h, w = ([pos[0]], [pos[1]], [pos[2]])
+    return O.rope3d(x, 1, t, h, w, split, theta)[0, 0]
+
+
+def test_rope_pos0_is_identity():
+    x = rng(1).standard_normal((5, 3, 128))
+    y = O.rope3d(x, 5, [0] * 5, [0] * 5, [0] * 5)
+    assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("split,theta,unit_pos", [
+    ((32, 48, 48), 10000.0, 100),   # theta^(-1/2) = 1/100: pos 100 -> 1 rad
+    ((16, 56, 56), 256.0, 16),      # page's split and base: 256^(-1/2) = 1/16
+])
+def test_rope_quarter_pair_turns_one_radian(split, theta, unit_pos):
+    """Pair j = d_a/4 of each axis chunk has frequency theta^(-1/2)."""
+    d_t, d_h, d_w = split
+    offs = (0, d_t, d_t + d_h)
+    for axis, d_a in enumerate(split):
+        dim = offs[axis] + 2 * (d_a // 4)
+        vec = np.zeros(128)
+        vec[dim] = 1.0
+        pos = [0, 0, 0]
+        pos[axis] = unit_pos
+        y = _one_token(vec, pos, split, theta)
+        assert y[dim] == pytest.approx(COS1, abs=1e-15)
+        assert y[dim + 1] == pytest.approx(SIN1, abs=1e-15)
+        others = np.delete(y, [dim, dim + 1])
+        assert np.all(others == 0.0)
+
+
+def test_rope_first_pair_turns_pos_radians_and_sign():
+    # Pair 0 has frequency 1: position 1 turns (1, 0) to (cos 1, sin 1) and
+    # (0, 1) to (-sin 1, cos 1): a counter-clockwise rotation.
+    for axis, off in enumerate((0, 32, 80)):
+        pos = [0, 0, 0]
+        pos[axis] = 1
+        e0 = np.zeros(128); e0[off] = 1.0
+        e1 = np.zeros(128); e1[off + 1] = 1.0
+        y0 = _one_token(e0, pos, (32, 48, 48), 10000.0)
+        y1 = _one_token(e1, pos, (32, 48, 48), 10000.0)
+        assert y0[off] == pytest.approx(COS1, abs=1e-15)
+        assert y0[off + 1] == pytest.approx(SIN1, abs=1e-15)
+        assert y1[off] == pytest.approx(-SIN1, abs=1e-15)
+        assert y1[off + 1] == pytest.approx(COS1, abs=1e-15)
+
+
+def test_rope_axis_isolation():
+    x = rng(2).standard_normal(128)
+    for axis, (lo, hi) in enumerate(((0, 32), (32, 80), (80, 128))):
+        pos = [0, 0, 0]
+        pos[axis] = 7
+        y = _one_token(x, pos, (32, 48, 48), 10000.0)
+        changed = np.nonzero(y != x)[0]
+        assert changed.min() >= lo and changed.max() < hi
+        assert changed.size == hi - lo
+
+
+def test_rope_preserves_pair_norms():
+    r = rng(3)
+    x = r.standard_normal((40, 4, 128))
+    t, h, w = r.integers(0, 500, (3, 40))
+    y = O.rope3d(x, 40, t, h, w)
+    nx = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    ny = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    assert np.allclose(nx, ny, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_dot_product_depends_only_on_position_difference():
+    r = rng(4)
+    q = r.standard_normal((1, 1, 128))
+    k = r.standard_normal((1, 1, 128))
+    p = r.integers(0, 300, 3)
+    pk = r.integers(0, 300, 3)
+
+    def dot(a, b):
+        rq = O.rope3d(q, 1, [a[0]], [a[1]], [a[2]])
+        rk = O.rope3d(k, 1, [b[0]], [b[1]], [b[2]])
+        return float(np.sum(rq * rk))
+
+    base = dot(p, pk)
+    for c in (np.array([3, 0, 0]), np.array([0, 11, 0]), np.array([0, 0, 29]),
+              np.array([41, 5, 17])):
+        assert dot(p + c, pk + c) == pytest.approx(base, rel=1e-10, abs=1e-10)
+    # ... and does depend on the difference.
+    assert abs(dot(p + np.array([0, 0, 1]), pk) - base) > 1e-6
+
+
+def test_rope_single_axis_is_complex_multiplication():
+    """1-D case in the textbook complex form: z_j -> z_j * e^{i pos w_j}."""
+    r = rng(5)
+    x = r.standard_normal(128)
+    pos = 37
+    y = _one_token(x, [pos, 0, 0], (32, 48, 48), 10000.0)
+    z = x[0:32:2] + 1j * x[1:32:2]
+    zj = z * np.exp(1j * pos * 10000.0 ** (-np.arange(16) / 16.0))
+    assert np.allclose(y[0:32:2], zj.real, atol=1e-12)
+    assert np.allclose(y[1:32:2], zj.imag, atol=1e-12)
+
+
+def test_rope_text_rows_unchanged():
+    x = rng(6).standard_normal((10, 2, 128))
+    y = O.rope3d(x, 4, [3] * 10, [2] * 10, [1] * 10)
+    assert np.array_equal(x[4:], y[4:])
+    assert not np.array_equal(x[:4], y[:4])
+
+
+# --------------------------------------------------- append and select -----
+def test_append_writes_rows_and_keeps_the_rest():
+    ck = np.arange(10 * 2 * 4, dtype=np.uint16).reshape(10, 2, 4)
+    cv = ck + 1000
+    kn = np.full((3, 2, 4), 7, dtype=np.uint16)
+    vn = np.full((3, 2, 4), 9, dtype=np.uint16)
+    k2, v2, n = O.kvcache_append(ck, cv, 4, kn, vn)
+    assert n == 7
+    assert np.all(k2[4:7] == 7) and np.all(v2[4:7] == 9)
+    assert np.array_equal(k2[:4], ck[:4]) and np.array_equal(k2[7:], ck[7:])
+    assert np.array_equal(v2[:4], cv[:4]) and np.array_equal(v2[7:], cv[7:])
+    with pytest.raises(ValueError):
+        O.kvcache_append(ck, cv, 8, kn, vn)
+
+
+def test_select_hand_example():
+    # 3 frames of 2 tokens; token rows hold their own index.
+    src = np.arange(6, dtype=np.uint16).reshape(6, 1, 1)
+    win = O.kvcache_select(src, [2, 0, 2, 1], tokens_per_frame=2)
+    assert win.ravel().tolist() == [4, 5, 0, 1, 4, 5, 2, 3]
+    with pytest.raises(IndexError):
+        O.kvcache_select(src, [3], 2)
+    with pytest.raises(IndexError):
+        O.kvcache_select(src, [-1], 2)
+    assert O.kvcache_select(src, [], 2).shape == (0, 1, 1)
+
+
+def test_cache_row_bytes_match_pages(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "cache_sizes.json")))
+    row = g["heads"] * g["head_dim"] * 2          # one bf16 K (or V) row
+    assert g["heads"] * g["head_dim"] == g["hidden"]
+    assert 2 * row == g["bf16_bytes_per_token_layer"]
+    assert 2 * row * g["layers"] == g["bf16_bytes_per_token_all_layers"]
+    per_frame = 2 * row * g["layers"] * g["tokens_per_frame_720p"]
+    assert round(per_frame / 1e6) == g["bf16_megabytes_per_frame_all_layers"]
+    int8 = 2 * (g["hidden"] + 4 * g["heads"])
+    assert int8 == g["int8_bytes_per_token_layer"]
+
+
+# ------------------------------------------------------------ attention ----
+def brute_force_attention(q, k, v, scale):
+    """Plain loops, naive exp with no max subtraction (tiny inputs only)."""
+    nq, nh, d = q.shape
+    nk = k.shape[0]
+    out = np.zeros_like(q)
+    lse = np.zeros((nh, nq))
+    for h in range(nh):
+        for i in range(nq):
+            w = []
+            for j in range(nk):
+                s = 0.0
+                for c in range(d):
+                    s += q[i, h, c] * k[j, h, c]
+                w.append(math.exp(s * scale))
+            z = sum(w)
+            for c in range(d):
+                out[i, h, c] = sum(w[j] * v[j, h, c] for j in range(nk)) / z
+            lse[h, i] = math.log(z)
+    return out, lse
+
+
+@pytest.mark.parametrize("nq,nk,nh,d", [(3, 5, 2, 8), (2, 13, 1, 16), (4, 16, 2, 128)])
+def test_attention_brute_force(nq, nk, nh, d):
+    r = rng(nq * 100 + nk)
+    q, k, v = (r.standard_normal((n, nh, d)) for n in (nq, nk, nk))
+    o, lse = O.attention(q, [(k, v)])
+    ob, lb = brute_force_attention(q, k, v, 1.0 / math.sqrt(d))
+    assert np.allclose(o, ob, atol=1e-12)
+    assert np.allclose(lse, lb, atol=1e-12)
+
+
+def test_attention_two_key_closed_form():
+    # q = sqrt(128) ln 3 e0, k1 = e0, k2 = 0: scores ln 3 and 0, so the
+    # weights are exactly 3/4 and 1/4 and LSE = ln(3 + 1).
+    d = 128
+    q = np.zeros((1, 1, d)); q[0, 0, 0] = math.sqrt(d) * math.log(3.0)
+    k = np.zeros((2, 1, d)); k[0, 0, 0] = 1.0
+    v = np.zeros((2, 1, d)); v[0, 0, 0] = 4.0; v[1, 0, 1] = 4.0
+    o, lse = O.attention(q, [(k, v)])
+    assert o[0, 0, 0] == pytest.approx(3.0, abs=1e-13)
+    assert o[0, 0, 1] == pytest.approx(1.0, abs=1e-13)
+    assert np.all(o[0, 0, 2:] == 0)
+    assert lse[0, 0] == pytest.approx(math.log(4.0), abs=1e-13)
+
+
+def test_attention_rows_sum_to_one():
+    r = rng(7)
+    q = 3 * r.standard_normal((9, 2, 128))
+    k = r.standard_normal((50, 2, 128))
+    o, _ = O.attention(q, [(k, np.ones_like(k))])
+    assert np.allclose(o, 1.0, atol=1e-13)
+
+
+def test_attention_zero_query_gives_mean_of_v():
+    r = rng(8)
+    k = r.standard_normal((33, 3, 128))
+    v = r.standard_normal((33, 3, 128))
+    o, lse = O.attention(np.zeros((2, 3, 128)), [(k, v)])
+    assert np.allclose(o, v.mean(axis=0)[None], atol=1e-13)
+    assert np.allclose(lse, math.log(33), atol=1e-13)
+
+
+def test_attention_split_equals_concatenation_and_lse_merge():
+    r = rng(9)
+    q = r.standard_normal((6, 2, 128))
+    ks = [r.standard_normal((n, 2, 128)) for n in (7, 3, 11)]
+    vs = [r.standard_normal((n, 2, 128)) for n in (7, 3, 11)]
+    o_split, l_split = O.attention(q, list(zip(ks, vs)))
+    o_cat, l_cat = O.attention(q, [(np.concatenate(ks), np.concatenate(vs))])
+    assert np.allclose(o_split, o_cat, atol=1e-13)
+    # Merging partial results: O = sum_p e^{LSE_p - LSE} O_p, LSE = ln sum e^LSE_p.
+    parts = [O.attention(q, [(k, v)]) for k, v in zip(ks, vs)]
+    lse = np.log(sum(np.exp(p[1]) for p in parts))
+    merged = sum(np.exp(p[1] - lse).T[:, :, None] * p[0] for p in parts)
+    assert np.allclose(merged, o_cat, atol=1e-12)
+    assert np.allclose(lse, l_cat, atol=1e-12)
+
+
+def test_attention_key_permutation_invariance():
+    r = rng(10)
+    q = r.standard_normal((4, 2, 128))
+    k = r.standard_normal((20, 2, 128))
+    v = r.standard_normal((20, 2, 128))
+    perm = r.permutation(20)
+    o1, l1 = O.attention(q, [(k, v)])
+    o2, l2 = O.attention(q, [(k[perm], v[perm])])
+    assert np.allclose(o1, o2, atol=1e-13) and np.allclose(l1, l2, atol=1e-13)
+
+
+def test_attention_one_hot_key_selects_its_value():
+    r = rng(11)
+    k = r.standard_normal((30, 1, 128))
+    v = r.standard_normal((30, 1, 128))
+    q = 40.0 * k[17:18] / np.linalg.norm(k[17])  # far larger score on key 17
+    o, _ = O.attention(q, [(k, v)])
+    assert np.allclose(o[0, 0], v[17, 0], atol=1e-6)
+
+
+def test_attention_large_scores_stay_finite():
+    # Scores of ~1e3: naive exp would overflow, the two-pass form must not.
+    r = rng(12)
+    k = r.standard_normal((8, 1, 128))
+    q = 1e3 * np.ones((1, 1, 128))
+    o, lse = O.attention(q, [(k, k)])
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+def test_attention_rows_subset_equals_full():
+    r = rng(13)
+    q = r.standard_normal((300, 2, 128))
+    k = r.standard_normal((40, 2, 128))
+    v = r.standard_normal((40, 2, 128))
+    o, l = O.attention(q, [(k, v)])
+    rows = np.array([0, 7, 255, 256, 299])
+    o2, l2 = O.attention_rows(q, rows, [(k, v)])
+    # Rows are independent; BLAS may block a different row count differently.
+    assert np.allclose(o[rows], o2, atol=1e-13) and np.allclose(l[:, rows], l2, atol=1e-13)
+
+
+def test_attention_no_keys():
+    o, l = O.attention(np.ones((2, 1, 8)), [(np.zeros((0, 1, 8)), np.zeros((0, 1, 8)))])
+    assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+# --------------------------------------------------------- frame picker ----
+def test_picker_printed_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "frame_picker_T360.json")))
+    got = O.temporal_context_frame_indices(g["n_past"], g["budget"], g["gamma"])
+    assert got.tolist() == g["kept_frames"]
+
+
+@pytest.mark.parametrize("t", [1, 2, 5, 17, 18])
+def test_picker_short_history_keeps_everything(t):
+    assert O.temporal_context_frame_indices(t).tolist() == list(range(t))
+
+
+@pytest.mark.parametrize("t", [19, 60, 361, 2000])
+def test_picker_keeps_first_and_newest_frames(t):
+    got = O.temporal_context_frame_indices(t)
+    assert got.size == 18 and got[0] == 0 and got[-1] == t - 1
+    assert np.all(np.diff(got) > 0)
+
+
+def test_picker_empty_history():
+    assert O.temporal_context_frame_indices(0).size == 0
