@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Segment-over-cache attention layer-step benchmark on B200.
+
+One step = one pass of the whole hot path over one layer's inputs, resident
+in HBM: fused RoPE-3D + cache append of the segment (rotated Q out, rotated K
+and V into the cache), for the bounded-history workload the frame-list gather
+of the history window, then segment attention of the segment + text queries
+over history + text + segment keys.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 720p]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
+
+Multi-GPU (torchrun): every rank runs its own independent layer-step (weak
+scaling, no collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "segment-over-cache attention TFLOP/s and % of B200 BF16 peak; ms per layer-step"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=40)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["nomas", "reference"], default="nomas")
+    p.add_argument("--workload", choices=["720p", "bounded", "mid", "tiny"], default="720p")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("attention.cu", "tmem_ops.cuh", "nomas_internal.h"):
+        with open(os.path.join(ROOT, "kv_cached_segment_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if the
+    kernel source has not changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"attention_{workload}_dram.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if uuid:
+                cmd += ["-i", uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[3:7]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- workload --
+class LayerStep:
+    """Device-resident buffers of one layer-step and the launches of a step."""
+
+    def __init__(self, wname: str, seed: int):
+        import torch
+
+        import kv_cached_segment_b200 as nm
+        from seeded_inputs import WORKLOADS, bounded_frame_list, randn_bf16
+
+        self.nm, self.torch = nm, torch
+        w = self.w = WORKLOADS[wname]
+        dev = "cuda"
+        ns, nt = w.n_seg, w.n_text
+        self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        self.cache = nm.KVCache.empty(w.n_cache + ns, w.tokens_per_frame)
+        self.cache.k[:w.n_cache] = randn_bf16((w.n_cache, 16, 128), seed * 16 + 4, dev)
+        self.cache.v[:w.n_cache] = randn_bf16((w.n_cache, 16, 128), seed * 16 + 5, dev)
+        self.q = randn_bf16((w.n_q, 16, 128), seed * 16 + 1, dev)
+        self.k = randn_bf16((w.n_q, 16, 128), seed * 16 + 2, dev)
+        self.v = randn_bf16((w.n_q, 16, 128), seed * 16 + 3, dev)
+        self.q_rot = torch.empty_like(self.q)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        if w.select_frames:
+            self.frames = bounded_frame_list(w, seed).tolist()
+            self.window = nm.KVCache.empty(w.n_window, 0)
+        else:
+            self.frames = None
+        self.launches_per_step = 3 if self.frames else 2
+
+    def flops(self) -> float:
+        return self.w.attention_flops()
+
+    def run(self, ev=None):
+        nm, w = self.nm, self.w
+        ns = w.n_seg
+        self.cache.len = w.n_cache
+        nm.kvcache_append(self.cache, self.k[:ns], self.v[:ns], q_in=self.q, q_out=self.q_rot,
+                          layout=self.layout, cfg=self.cfg)
+        if self.frames is not None:
+            nm.kvcache_select(self.cache, self.frames, self.window)
+            hist = self.window.span()
+        else:
+            hist = self.cache.span(0, w.n_cache)
+        spans = [hist, (self.k[ns:], self.v[ns:]), self.cache.span(w.n_cache, w.n_cache + ns)]
+        if ev is not None:
+            ev[0].record()
+        nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
+        if ev is not None:
+            ev[1].record()
+
+    def host_inputs(self):
+        """Pinned host copies of one step's inputs (for the end-to-end leg)."""
+        t = self.torch
+        return {n: getattr(self, n).cpu().pin_memory() for n in ("q", "k", "v")}, \
+            t.empty_like(self.o, device="cpu").pin_memory()
+
+
+def cpu_oracle_rate(step: LayerStep, budget_s: float, rows_per_chunk: int, max_rows: int):
+    """Times the fp64 oracle (RoPE of the sampled rows + their attention over
+    every key) on host cores; returns (TFLOP/s, rows, seconds, threads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    def f64(t):
+        b = t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+        return oracle.bf16_bits_to_f64(b)
+
+    w = step.w
+    ns = w.n_seg
+    hist_k = step.window.k[:w.n_window] if step.frames else step.cache.k[:w.n_cache]
+    hist_v = step.window.v[:w.n_window] if step.frames else step.cache.v[:w.n_cache]
+    spans = [(f64(hist_k), f64(hist_v)), (f64(step.k[ns:]), f64(step.v[ns:])),
+             (f64(step.k[:ns]), f64(step.v[:ns]))]
+    t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    q_all = step.q
+    rng = np.random.default_rng(0)
+    done, elapsed = 0, 0.0
+    t0 = time.perf_counter()
+    while elapsed < budget_s and done < max_rows:
+        rows = np.sort(rng.integers(0, ns, rows_per_chunk))
+        q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
+                               ww[rows])
+        k_seg = spans[2][0]
+        if done == 0:
+            k_seg = oracle.rope3d(k_seg, ns, t, h, ww)  # the segment's keys, once
+            spans[2] = (k_seg, spans[2][1])
+        oracle.attention(q_rows, spans)
+        done += rows.size
+        elapsed = time.perf_counter() - t0
+    flops = 4.0 * done * w.n_k * 128 * 16
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    return flops / elapsed / 1e12, done, elapsed, threads
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks, peak_src = load_peaks()
+    step = LayerStep(args.workload, seed=1 + rank)
+    torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize()
+    if int(step.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(step.err.item())}")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(local_rank).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:  # noqa: BLE001
+        uuid = None
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        step.run(evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+
+    ms = start.elapsed_time(stop)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    if world > 1:
+        t = torch.tensor([ms, attn_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, attn_ms = float(t[0]), float(t[1])
+    ms_per_step = ms / args.steps
+    flops = step.flops()
+    value = flops * args.steps * world / (ms / 1e3) / 1e12
+    attn_tflops = flops / (attn_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_in, host_o = step.host_inputs()
+        for _ in range(2):
+            run_e2e(step, host_in, host_o)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 20))
+        e0.record()
+        for _ in range(n_e2e):
+            run_e2e(step, host_in, host_o)
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+        e2e = {"value": flops * n_e2e * world / (e_ms / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": host_o.numel() * 2,
+               "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, rows, secs, threads = cpu_oracle_rate(step, budget_s=12.0, rows_per_chunk=16,
+                                                    max_rows=512)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 oracle RoPE + attention of {rows} sampled segment query rows "
+                         f"x 16 heads over all {step.w.n_k} keys ({secs:.1f} s)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    w = step.w
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: {w.frames}x{w.grid_h}x{w.grid_w} segment tokens + {w.n_text} "
+                        f"text over {w.n_window if w.select_frames else w.n_cache} history tokens",
+            "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
+            "attention_flops_per_step": flops,
+            "step": "fused rope3d+append" + (" + select" if w.select_frames else "")
+                    + " + segment attention",
+            "l2": "inputs larger than L2: each step reads "
+                  f"{(w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
+            "parallelism": f"independent layer-step per GPU x{world}",
+        },
+        "pct_of_measured_bf16_peak": 100.0 * value / peak,
+        "pct_of_datasheet_bf16_peak": 100.0 * value / DATASHEET_BF16_TFLOPS,
+        "attention_ms": attn_ms,
+        "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn_tflops,
+                     "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": recorded_traffic(args.workload)},
+        "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+
+
+def run_e2e(step: LayerStep, host_in, host_o):
+    step.q.copy_(host_in["q"], non_blocking=True)
+    step.k.copy_(host_in["k"], non_blocking=True)
+    step.v.copy_(host_in["v"], non_blocking=True)
+    step.run()
+    host_o.copy_(step.o, non_blocking=True)
+
+
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle as it stands, on the same workload, metric and unit."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from seeded_inputs import WORKLOADS, layer_inputs
+
+    w = WORKLOADS[args.workload]
+    inp = layer_inputs(w, seed=1)
+
+    def f64(t):
+        b = t.detach().contiguous().view(torch.int16).numpy().view(np.uint16)
+        return oracle.bf16_bits_to_f64(b)
+
+    ns = w.n_seg
+    t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    hist_k, hist_v = f64(inp["cache_k"]), f64(inp["cache_v"])
+    if w.select_frames:
+        from seeded_inputs import bounded_frame_list
+        idx = bounded_frame_list(w, 1)
+        hist_k = oracle.kvcache_select(hist_k, idx, w.tokens_per_frame)
+        hist_v = oracle.kvcache_select(hist_v, idx, w.tokens_per_frame)
+    k_seg = oracle.rope3d(f64(inp["k"][:ns]), ns, t, h, ww)
+    spans = [(hist_k, hist_v), (f64(inp["k"][ns:]), f64(inp["v"][ns:])), (k_seg, f64(inp["v"][:ns]))]
+    q_all = inp["q"]
+    rows_per_step = 8
+    rng = np.random.default_rng(0)
+
+    def one_step():
+        rows = np.sort(rng.integers(0, ns, rows_per_step))
+        q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
+                               ww[rows])
+        oracle.attention(q_rows, spans)
+
+    for _ in range(max(3, args.warmup)):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    secs = time.perf_counter() - t0
+    flops = 4.0 * rows_per_step * w.n_k * 128 * 16 * args.steps
+    value = flops / secs / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {rows_per_step} sampled segment query rows per step "
+                               f"x 16 heads over all {w.n_k} keys", "n_q": w.n_q, "n_k": w.n_k},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} query rows per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * nomas.h -- C ABI of libnomas, segment-over-cache attention for B200 (sm_100a).
+ *
+ * The operations are those of one attention layer of a segment-autoregressive
+ * video world model whose only memory is a per-layer KV cache of past
+ * segments:
+ *   "Hy-Nomas: an 8.6B world model whose memory is a KV cache"
+ *   (ai.thesatyajit.com), sections "How one segment is made", "Writing the
+ *   segment into memory", "What 'world memory' stores" and "The 4090 preset".
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE memory; the library never allocates,
+ *     frees or keeps a pointer after a call returns.
+ *   - bf16 values are passed as raw 16-bit patterns (void pointers).  Q, K, V
+ *     and O rows have layout [tokens][heads][head_dim], contiguous; a row of
+ *     16 x 128 bf16 is 4096 bytes.  Every tensor pointer must be 16-byte
+ *     aligned.
+ *   - Only heads = 16 and head_dim = 128 are implemented; other values return
+ *     NOMAS_ERR_UNSUPPORTED.
+ *   - Every call is asynchronous on the caller's stream (`stream` is a
+ *     cudaStream_t; NULL is the legacy default stream) and never synchronises.
+ *     Argument errors are detected on the host before anything is launched and
+ *     leave all memory untouched.
+ *   - Errors found on the device (a bad index in a device-resident frame list,
+ *     a pipeline wait that exceeded its time limit) never trap: the kernel
+ *     ORs a NOMAS_DEVERR_* bit into the caller's optional int32 word
+ *     `dev_err` (device memory) and skips the affected work.  The caller
+ *     reads the word after synchronising.
+ *   - nomas_last_error() returns a per-thread message for the last failing
+ *     call made by that thread.
+ */
+#ifndef NOMAS_H
+#define NOMAS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NOMAS_OK = 0,
+  NOMAS_ERR_INVALID_ARG = 1, /* NULL / misaligned pointer, bad size or layout */
+  NOMAS_ERR_CAPACITY = 2,    /* a write would run past a cache's capacity     */
+  NOMAS_ERR_INDEX = 3,       /* a host frame index outside the source cache   */
+  NOMAS_ERR_UNSUPPORTED = 4, /* heads != 16 or head_dim != 128, too many spans */
+  NOMAS_ERR_CUDA = 5         /* a CUDA runtime/driver call failed             */
+} nomas_status;
+
+/* Bits ORed into *dev_err by kernels. */
+#define NOMAS_DEVERR_BAD_FRAME_INDEX 0x1 /* select: device list entry out of range */
+#define NOMAS_DEVERR_WAIT_TIMEOUT 0x2    /* attention: a pipeline wait timed out   */
+
+#define NOMAS_HEADS 16
+#define NOMAS_HEAD_DIM 128
+#define NOMAS_MAX_SPANS 4
+
+/*
+ * 3D rotary configuration: the head dimension is split into a temporal chunk
+ * of d_t dims, a grid-row chunk of d_h dims and a grid-column chunk of d_w
+ * dims (d_t + d_h + d_w = head_dim, each even and > 0); pair j of a chunk of
+ * width d turns by pos * theta^(-2j/d) radians.  Pairs are adjacent elements
+ * (2j, 2j+1) inside the chunk.  The page's own values are d = 16/56/56 and
+ * theta = 256 ("How one segment is made", item "The blocks"); 32/48/48 with
+ * theta = 10000 is the default of the measured workloads.
+ */
+typedef struct {
+  int32_t d_t, d_h, d_w;
+  float theta;
+} nomas_rope3d_cfg;
+
+/*
+ * Row layout of one segment: `frames * grid_h * grid_w` video rows first
+ * (frame-major, then row-major over the latent grid; one token per grid cell,
+ * "How one segment is made", items "Video tokens" and "The blocks"), then
+ * `n_text` text rows.  Video row r sits at t = t0 + r / (grid_h*grid_w),
+ * h = (r / grid_w) % grid_h, w = r % grid_w; t0 is the number of latent
+ * frames already written to the history, so positions continue across
+ * segments.  Text rows carry no 3D position and are not rotated.
+ */
+typedef struct {
+  int32_t frames, grid_h, grid_w, t0, n_text;
+} nomas_seg_layout;
+
+/*
+ * One layer's KV cache ("What 'world memory' stores"): K and V each hold
+ * `capacity` rows of [heads][head_dim] bf16; rows [0, len) are valid.  A
+ * latent frame is `tokens_per_frame` consecutive rows.  Keys are stored
+ * after rotation, so a frame keeps its original position when it is later
+ * gathered into a window.  The struct is host memory owned by the caller;
+ * k and v point to device memory owned by the caller.
+ */
+typedef struct {
+  void *k, *v;
+  int64_t capacity, len;
+  int32_t tokens_per_frame, heads, head_dim;
+} nomas_kvcache;
+
+/* A contiguous run of `len` key/value rows ([len][heads][head_dim] bf16). */
+typedef struct {
+  const void *k, *v;
+  int64_t len;
+} nomas_kv_span;
+
+/* Message describing the last failing call on this host thread ("" if none). */
+const char *nomas_last_error(void);
+
+/* Library version string. */
+const char *nomas_version(void);
+
+/*
+ * 3D RoPE on Q and K ("How one segment is made", item "The blocks": 3D RoPE
+ * over (t, h, w)).
+ *   q, k       : [n][heads][head_dim] bf16 inputs, n = video rows + n_text.
+ *                k may be NULL (then k_out must be NULL): Q only.
+ *   q_out,k_out: outputs of the same shape; may equal the inputs (in place),
+ *                must not otherwise overlap them.  Text rows are copied.
+ *   layout     : row layout (host struct); cfg: rotary configuration (host).
+ * Rotation is fp32 arithmetic on the widened bf16 inputs with angles and their
+ * cosines/sines evaluated in double, rounded to bf16 to nearest-even.
+ * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_rope3d_qk(const void *q, const void *k, void *q_out, void *k_out,
+                             const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
+                             int32_t heads, int32_t head_dim, void *stream);
+
+/*
+ * Segment write-back into the cache, fused with 3D RoPE ("Writing the
+ * segment into memory": after a segment is generated its keys and values are
+ * stored in the cache; "What 'world memory' stores": the cache grows by one
+ * segment per step).
+ *   cache   : host struct; rows [len, len + n_tokens) of cache->k receive the
+ *             rotated segment keys, the same rows of cache->v the values bit
+ *             for bit; every other row is left untouched.  On success
+ *             cache->len += n_tokens.
+ *   k_seg, v_seg: [n_tokens][heads][head_dim] bf16, the segment's video rows.
+ *   q_in, q_out : optional (both NULL, or both set): the segment's Q,
+ *             [n_tokens + layout->n_text][heads][head_dim]; video rows are
+ *             rotated into q_out, text rows copied (q_out may equal q_in).
+ *   layout  : required when cfg != NULL; then n_tokens must equal
+ *             frames * grid_h * grid_w.
+ *   cfg     : NULL -> plain copy of K and V (and Q), no rotation.
+ * Errors: NOMAS_ERR_CAPACITY if len + n_tokens > capacity (nothing written,
+ * len unchanged); NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_kvcache_append(nomas_kvcache *cache, const void *k_seg, const void *v_seg,
+                                  int64_t n_tokens, const void *q_in, void *q_out,
+                                  const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
+                                  void *stream);
+
+/*
+ * Bounded active history: gather whole latent frames of `src` into the
+ * contiguous `window` ("The 4090 preset": before each segment only a list of
+ * past latent frames is restored to the GPU).  Window rows
+ * [j*P, (j+1)*P) receive source rows [idx[j]*P, (idx[j]+1)*P), P =
+ * src->tokens_per_frame, for K and V, bit for bit.  Repeats are allowed.
+ *   frame_idx     : int32[n_frames], host memory if idx_on_device == 0, device
+ *                   memory otherwise.
+ *   window        : host struct; needs capacity >= n_frames * P and the same
+ *                   heads/head_dim; its tokens_per_frame is set to P and, on
+ *                   success, its len to n_frames * P.
+ *   dev_err       : device int32, required when idx_on_device != 0.
+ * A host index outside [0, src->len / P) returns NOMAS_ERR_INDEX before any
+ * launch.  A bad device index sets NOMAS_DEVERR_BAD_FRAME_INDEX in *dev_err
+ * and its window rows are left untouched; the other frames are copied.
+ * Errors: NOMAS_ERR_INDEX, NOMAS_ERR_CAPACITY, NOMAS_ERR_INVALID_ARG,
+ * NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame_idx,
+                                  int32_t n_frames, int32_t idx_on_device, nomas_kvcache *window,
+                                  int32_t *dev_err, void *stream);
+
+/*
+ * Segment-over-cache attention ("How one segment is made": joint attention
+ * of text and video tokens, causal across segments so the current segment
+ * reads earlier ones from the KV cache; "What 'world memory' stores": the
+ * queries of segment k attend over the cache).  Every query row attends to
+ * every key of every span with no mask:
+ *   O[i,h] = sum_j softmax_j(scale * <q[i,h], k[j,h]>) v[j,h]
+ *   LSE[h,i] = ln sum_j exp(scale * <q[i,h], k[j,h]>)
+ *   q      : [n_q][heads][head_dim] bf16 (already rotated).
+ *   spans  : host array of n_spans (1..NOMAS_MAX_SPANS) key/value runs, e.g.
+ *            cache (or window), text, segment; len 0 spans are skipped.
+ *   o      : [n_q][heads][head_dim] bf16 output, must not overlap inputs.
+ *   lse    : optional fp32 [heads][n_q] output (natural log); NULL to skip.
+ *   softmax_scale: <= 0 selects 1/sqrt(head_dim).
+ *   dev_err: optional device int32 (see the conventions above).
+ * With no keys at all, O = 0 and LSE = -inf.  bf16 operands, fp32 scores,
+ * softmax and accumulation; O rounded to bf16 to nearest-even.
+ * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                     int32_t n_spans, void *o, float *lse, float softmax_scale,
+                                     int32_t heads, int32_t head_dim, int32_t *dev_err,
+                                     void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NOMAS_H */

@@ -1,0 +1,279 @@
+"""Python binding of libnomas (segment-over-cache attention for B200).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels behind the C ABI declared in ``include/nomas.h``.  PyTorch provides
+device memory and streams.  There is no CPU fallback: if the compiled
+library is missing, importing the binding's entry points raises.
+
+Entry points (same names as the C ABI, without the ``nomas_`` prefix):
+``rope3d_qk``, ``kvcache_append``, ``kvcache_select``, ``segment_attention``,
+plus the ``KVCache`` holder and the ``RopeConfig`` / ``SegLayout`` structs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from . import _build
+
+HEADS = 16
+HEAD_DIM = 128
+
+NOMAS_OK = 0
+NOMAS_ERR_INVALID_ARG = 1
+NOMAS_ERR_CAPACITY = 2
+NOMAS_ERR_INDEX = 3
+NOMAS_ERR_UNSUPPORTED = 4
+NOMAS_ERR_CUDA = 5
+DEVERR_BAD_FRAME_INDEX = 0x1
+DEVERR_WAIT_TIMEOUT = 0x2
+MAX_SPANS = 4
+
+EXPORTED_SYMBOLS = (
+    "nomas_last_error",
+    "nomas_version",
+    "nomas_rope3d_qk",
+    "nomas_kvcache_append",
+    "nomas_kvcache_select",
+    "nomas_segment_attention",
+)
+
+
+class NomasError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"nomas status {status}: {message}")
+        self.status = status
+
+
+class _RopeCfg(ctypes.Structure):
+    _fields_ = [("d_t", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_w", ctypes.c_int32),
+                ("theta", ctypes.c_float)]
+
+
+class _SegLayout(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int32), ("grid_h", ctypes.c_int32),
+                ("grid_w", ctypes.c_int32), ("t0", ctypes.c_int32), ("n_text", ctypes.c_int32)]
+
+
+class _KVCache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("len", ctypes.c_int64), ("tokens_per_frame", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class _KVSpan(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Loads libnomas.so (built in-tree by ``_build.build``); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or _build.LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m kv_cached_segment_b200._build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    lib.nomas_last_error.restype = ctypes.c_char_p
+    lib.nomas_last_error.argtypes = []
+    lib.nomas_version.restype = ctypes.c_char_p
+    lib.nomas_version.argtypes = []
+    lib.nomas_rope3d_qk.restype = ctypes.c_int
+    lib.nomas_rope3d_qk.argtypes = [P, P, P, P, ctypes.POINTER(_SegLayout),
+                                    ctypes.POINTER(_RopeCfg), I32, I32, P]
+    lib.nomas_kvcache_append.restype = ctypes.c_int
+    lib.nomas_kvcache_append.argtypes = [ctypes.POINTER(_KVCache), P, P, I64, P, P,
+                                         ctypes.POINTER(_SegLayout), ctypes.POINTER(_RopeCfg), P]
+    lib.nomas_kvcache_select.restype = ctypes.c_int
+    lib.nomas_kvcache_select.argtypes = [ctypes.POINTER(_KVCache), P, I32, I32,
+                                         ctypes.POINTER(_KVCache), P, P]
+    lib.nomas_segment_attention.restype = ctypes.c_int
+    lib.nomas_segment_attention.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, F32,
+                                            I32, I32, P, P]
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != NOMAS_OK:
+        raise NomasError(status, load_library().nomas_last_error().decode())
+
+
+@dataclass
+class RopeConfig:
+    """3D rotary split of the head dimension over (t, h, w) and its base."""
+    d_t: int = 32
+    d_h: int = 48
+    d_w: int = 48
+    theta: float = 10000.0
+
+    def _c(self):
+        return _RopeCfg(self.d_t, self.d_h, self.d_w, self.theta)
+
+
+@dataclass
+class SegLayout:
+    """Video rows (frames x grid_h x grid_w, first latent frame at t0), then text rows."""
+    frames: int
+    grid_h: int
+    grid_w: int
+    t0: int
+    n_text: int
+
+    @property
+    def n_video(self) -> int:
+        return self.frames * self.grid_h * self.grid_w
+
+    def _c(self):
+        return _SegLayout(self.frames, self.grid_h, self.grid_w, self.t0, self.n_text)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _rows(t: torch.Tensor, name: str) -> int:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous CUDA bf16 tensor")
+    if t.dim() != 3 or t.shape[1] != HEADS or t.shape[2] != HEAD_DIM:
+        raise ValueError(f"{name} must have shape [N][{HEADS}][{HEAD_DIM}], got {tuple(t.shape)}")
+    return t.shape[0]
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class KVCache:
+    """One layer's KV cache: caller-owned K/V buffers of ``capacity`` rows, ``len`` valid."""
+
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, length: int, tokens_per_frame: int):
+        _rows(k, "cache k")
+        _rows(v, "cache v")
+        if k.shape != v.shape:
+            raise ValueError("cache k and v differ in shape")
+        self.k, self.v = k, v
+        self._c = _KVCache(k.data_ptr(), v.data_ptr(), k.shape[0], int(length),
+                           int(tokens_per_frame), HEADS, HEAD_DIM)
+
+    @classmethod
+    def empty(cls, capacity: int, tokens_per_frame: int, device="cuda"):
+        k = torch.empty((capacity, HEADS, HEAD_DIM), dtype=torch.bfloat16, device=device)
+        v = torch.empty_like(k)
+        return cls(k, v, 0, tokens_per_frame)
+
+    @property
+    def len(self) -> int:
+        return self._c.len
+
+    @len.setter
+    def len(self, n: int) -> None:
+        self._c.len = int(n)
+
+    @property
+    def capacity(self) -> int:
+        return self._c.capacity
+
+    @property
+    def tokens_per_frame(self) -> int:
+        return self._c.tokens_per_frame
+
+    def span(self, start: int = 0, stop: int | None = None):
+        """(k, v) views of rows [start, stop) (default: the valid rows)."""
+        stop = self.len if stop is None else stop
+        return self.k[start:stop], self.v[start:stop]
+
+
+def rope3d_qk(q, k, q_out, k_out, layout: SegLayout, cfg: RopeConfig, stream=None) -> None:
+    """3D RoPE on Q (and K): video rows rotated, text rows copied."""
+    lib = load_library()
+    n = _rows(q, "q")
+    _rows(q_out, "q_out")
+    if k is not None:
+        _rows(k, "k")
+        _rows(k_out, "k_out")
+    if n != layout.n_video + layout.n_text:
+        raise ValueError("q rows != video rows + text rows")
+    lay, c = layout._c(), cfg._c()
+    _check(lib.nomas_rope3d_qk(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), ctypes.byref(lay),
+                               ctypes.byref(c), HEADS, HEAD_DIM, _stream(stream)))
+
+
+def kvcache_append(cache: KVCache, k_seg, v_seg, q_in=None, q_out=None,
+                   layout: SegLayout | None = None, cfg: RopeConfig | None = None,
+                   stream=None) -> None:
+    """Rotates the segment's K into the cache (V copied), optionally Q too; advances len."""
+    lib = load_library()
+    n = _rows(k_seg, "k_seg")
+    if _rows(v_seg, "v_seg") != n:
+        raise ValueError("k_seg and v_seg differ in rows")
+    if q_in is not None:
+        _rows(q_in, "q_in")
+        _rows(q_out, "q_out")
+    lay = layout._c() if layout is not None else None
+    c = cfg._c() if cfg is not None else None
+    _check(lib.nomas_kvcache_append(ctypes.byref(cache._c), _ptr(k_seg), _ptr(v_seg), n,
+                                    _ptr(q_in), _ptr(q_out),
+                                    ctypes.byref(lay) if lay is not None else None,
+                                    ctypes.byref(c) if c is not None else None,
+                                    _stream(stream)))
+
+
+def kvcache_select(src: KVCache, frame_idx, window: KVCache, dev_err=None, stream=None) -> None:
+    """Gathers the listed latent frames of ``src`` into ``window`` (bit-exact)."""
+    lib = load_library()
+    if isinstance(frame_idx, torch.Tensor) and frame_idx.is_cuda:
+        if frame_idx.dtype != torch.int32 or not frame_idx.is_contiguous():
+            raise TypeError("device frame_idx must be contiguous int32")
+        n, on_dev, keep = frame_idx.numel(), 1, frame_idx
+        ptr = frame_idx.data_ptr()
+    else:
+        arr = (ctypes.c_int32 * len(frame_idx))(*[int(x) for x in frame_idx])
+        n, on_dev, keep = len(frame_idx), 0, arr
+        ptr = ctypes.cast(arr, ctypes.c_void_p).value
+    if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
+        raise TypeError("dev_err must be a CUDA int32 tensor")
+    _check(lib.nomas_kvcache_select(ctypes.byref(src._c), ptr, n, on_dev, ctypes.byref(window._c),
+                                    _ptr(dev_err), _stream(stream)))
+    del keep
+
+
+def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, dev_err=None,
+                      stream=None):
+    """Attention of every row of q over all keys of ``spans`` (list of (k, v)); returns o."""
+    lib = load_library()
+    n_q = _rows(q, "q")
+    if o is None:
+        o = torch.empty_like(q)
+    _rows(o, "o")
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_cuda or
+                            lse.numel() != HEADS * n_q or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous CUDA fp32 tensor of heads * n_q elements")
+    if len(spans) > MAX_SPANS:
+        raise ValueError(f"at most {MAX_SPANS} spans")
+    arr = (_KVSpan * max(1, len(spans)))()
+    for i, (k, v) in enumerate(spans):
+        nk = _rows(k, f"span {i} k")
+        if _rows(v, f"span {i} v") != nk:
+            raise ValueError(f"span {i}: k and v differ in rows")
+        arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
+    if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
+        raise TypeError("dev_err must be a CUDA int32 tensor")
+    _check(lib.nomas_segment_attention(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
+                                       float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
+                                       _stream(stream)))
+    return o

@@ -1,0 +1,381 @@
+// C-ABI entry points of libnomas (declared in include/nomas.h).
+//
+// Host side only: argument validation, tensor-map (TMA descriptor) encoding
+// and kernel launches.  Every check happens before anything is launched, so a
+// rejected call leaves device memory untouched.  Nothing here allocates
+// device memory, synchronises or keeps a caller pointer past the call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "nomas.h"
+#include "nomas_internal.h"
+
+using namespace nomas;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+nomas_status fail(nomas_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+nomas_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(NOMAS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+nomas_status ok() {
+  g_last_error.clear();
+  return NOMAS_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// [a, a + an) and [b, b + bn) overlap (bytes).
+bool overlap(const void *a, int64_t an, const void *b, int64_t bn) {
+  if (a == nullptr || b == nullptr || an <= 0 || bn <= 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + (uintptr_t)bn && y < x + (uintptr_t)an;
+}
+
+nomas_status check_shape(int32_t heads, int32_t head_dim) {
+  if (heads != kHeads || head_dim != kHeadDim)
+    return fail(NOMAS_ERR_UNSUPPORTED, "only heads=16, head_dim=128 are implemented (got %d, %d)",
+                heads, head_dim);
+  return NOMAS_OK;
+}
+
+nomas_status check_layout(const nomas_seg_layout *l, int64_t *n_video) {
+  if (l == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "layout is NULL");
+  if (l->frames < 0 || l->grid_h < 0 || l->grid_w < 0 || l->n_text < 0 || l->t0 < 0)
+    return fail(NOMAS_ERR_INVALID_ARG, "layout fields must be >= 0");
+  *n_video = (int64_t)l->frames * l->grid_h * l->grid_w;
+  if (*n_video > ((int64_t)1 << 31) || l->t0 > (1 << 30))
+    return fail(NOMAS_ERR_INVALID_ARG, "layout too large");
+  return NOMAS_OK;
+}
+
+// Fills the per-pair frequency and axis tables of a rotary configuration.
+nomas_status fill_rope(const nomas_rope3d_cfg *cfg, RopeArgs *a) {
+  if (cfg == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "rope cfg is NULL");
+  const int d[3] = {cfg->d_t, cfg->d_h, cfg->d_w};
+  for (int i = 0; i < 3; ++i)
+    if (d[i] <= 0 || (d[i] & 1))
+      return fail(NOMAS_ERR_INVALID_ARG, "rope split entries must be even and > 0 (%d, %d, %d)",
+                  d[0], d[1], d[2]);
+  if (d[0] + d[1] + d[2] != kHeadDim)
+    return fail(NOMAS_ERR_INVALID_ARG, "rope split must sum to head_dim=128 (%d+%d+%d)", d[0],
+                d[1], d[2]);
+  if (!(cfg->theta > 0.f) || !std::isfinite(cfg->theta))
+    return fail(NOMAS_ERR_INVALID_ARG, "rope theta must be finite and > 0");
+  const double theta = (double)cfg->theta;
+  for (int p = 0; p < kHeadDim / 2; ++p) {
+    int ax, j;
+    if (2 * p < d[0]) {
+      ax = 0;
+      j = p;
+    } else if (2 * p < d[0] + d[1]) {
+      ax = 1;
+      j = p - d[0] / 2;
+    } else {
+      ax = 2;
+      j = p - (d[0] + d[1]) / 2;
+    }
+    a->axis[p] = (int8_t)ax;
+    a->omega[p] = std::pow(theta, -2.0 * (double)j / (double)d[ax]);
+  }
+  return NOMAS_OK;
+}
+
+// cuTensorMapEncodeTiled, reached through the runtime so the library does not
+// link libcuda directly.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D view of a [rows][16][128] bf16 tensor: inner extent 2048 elements, row
+// pitch 4096 B; box = 64 elements (128 B, one swizzle span) x 128 rows.
+nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {(cuuint64_t)kRowElems, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NOMAS_OK;
+}
+
+unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s per pipeline wait
+
+}  // namespace
+
+extern "C" {
+
+const char *nomas_last_error(void) { return g_last_error.c_str(); }
+
+const char *nomas_version(void) { return "nomas 0.1.0 (sm_100a)"; }
+
+nomas_status nomas_rope3d_qk(const void *q, const void *k, void *q_out, void *k_out,
+                             const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
+                             int32_t heads, int32_t head_dim, void *stream) {
+  nomas_status st = check_shape(heads, head_dim);
+  if (st != NOMAS_OK) return st;
+  int64_t n_video = 0;
+  if ((st = check_layout(layout, &n_video)) != NOMAS_OK) return st;
+  RopeArgs a{};
+  if ((st = fill_rope(cfg, &a)) != NOMAS_OK) return st;
+  const int64_t n = n_video + layout->n_text;
+  if (q == nullptr || q_out == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "q and q_out are required");
+  if ((k == nullptr) != (k_out == nullptr))
+    return fail(NOMAS_ERR_INVALID_ARG, "k and k_out must both be set or both be NULL");
+  if (!aligned16(q) || !aligned16(q_out) || !aligned16(k) || !aligned16(k_out))
+    return fail(NOMAS_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const int64_t bytes = n * kRowBytes;
+  if (q_out != q && overlap(q, bytes, q_out, bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_out partially overlaps q");
+  if (k != nullptr && k_out != k && overlap(k, bytes, k_out, bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "k_out partially overlaps k");
+  if (k != nullptr && (overlap(q_out, bytes, k_out, bytes) || overlap(q_out, bytes, k, bytes) ||
+                       overlap(k_out, bytes, q, bytes)))
+    return fail(NOMAS_ERR_INVALID_ARG, "Q and K buffers overlap");
+  a.q_in = static_cast<const uint16_t *>(q);
+  a.q_out = static_cast<uint16_t *>(q_out);
+  a.k_in = static_cast<const uint16_t *>(k);
+  a.k_out = static_cast<uint16_t *>(k_out);
+  a.n_q_rows = n;
+  a.n_kv_rows = k != nullptr ? n : 0;
+  a.n_video = n_video;
+  a.grid_h = layout->grid_h;
+  a.grid_w = layout->grid_w;
+  a.t0 = layout->t0;
+  if (n == 0) return ok();
+  const cudaError_t e = launch_rope_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rope3d launch");
+  return ok();
+}
+
+nomas_status nomas_kvcache_append(nomas_kvcache *cache, const void *k_seg, const void *v_seg,
+                                  int64_t n_tokens, const void *q_in, void *q_out,
+                                  const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
+                                  void *stream) {
+  if (cache == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "cache is NULL");
+  nomas_status st = check_shape(cache->heads, cache->head_dim);
+  if (st != NOMAS_OK) return st;
+  if (cache->k == nullptr || cache->v == nullptr || !aligned16(cache->k) || !aligned16(cache->v))
+    return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
+  if (cache->capacity < 0 || cache->len < 0 || cache->len > cache->capacity)
+    return fail(NOMAS_ERR_INVALID_ARG, "cache len/capacity inconsistent (%lld/%lld)",
+                (long long)cache->len, (long long)cache->capacity);
+  if (n_tokens < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_tokens < 0");
+  if (n_tokens > 0 && (k_seg == nullptr || v_seg == nullptr))
+    return fail(NOMAS_ERR_INVALID_ARG, "k_seg and v_seg are required");
+  if ((q_in == nullptr) != (q_out == nullptr))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_in and q_out must both be set or both be NULL");
+  if (!aligned16(k_seg) || !aligned16(v_seg) || !aligned16(q_in) || !aligned16(q_out))
+    return fail(NOMAS_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  RopeArgs a{};
+  int64_t n_video = 0, n_text = 0;
+  if (layout != nullptr) {
+    if ((st = check_layout(layout, &n_video)) != NOMAS_OK) return st;
+    n_text = layout->n_text;
+  }
+  if (cfg != nullptr) {
+    if (layout == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "rope cfg given without a layout");
+    if ((st = fill_rope(cfg, &a)) != NOMAS_OK) return st;
+    if (n_video != n_tokens)
+      return fail(NOMAS_ERR_INVALID_ARG, "n_tokens (%lld) != frames*grid_h*grid_w (%lld)",
+                  (long long)n_tokens, (long long)n_video);
+  }
+  if (cache->len + n_tokens > cache->capacity)
+    return fail(NOMAS_ERR_CAPACITY, "append of %lld rows at len %lld exceeds capacity %lld",
+                (long long)n_tokens, (long long)cache->len, (long long)cache->capacity);
+  const int64_t q_rows = q_in != nullptr ? n_tokens + n_text : 0;
+  uint16_t *k_dst = static_cast<uint16_t *>(cache->k) + cache->len * kRowElems;
+  uint16_t *v_dst = static_cast<uint16_t *>(cache->v) + cache->len * kRowElems;
+  const int64_t seg_bytes = n_tokens * kRowBytes, q_bytes = q_rows * kRowBytes;
+  if (overlap(k_seg, seg_bytes, k_dst, seg_bytes) || overlap(v_seg, seg_bytes, v_dst, seg_bytes) ||
+      overlap(k_seg, seg_bytes, v_dst, seg_bytes) || overlap(v_seg, seg_bytes, k_dst, seg_bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "segment K/V overlap the cache rows being written");
+  if (q_in != nullptr && q_out != q_in && overlap(q_in, q_bytes, q_out, q_bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_out partially overlaps q_in");
+  if (q_out != nullptr && (overlap(q_out, q_bytes, k_dst, seg_bytes) ||
+                           overlap(q_out, q_bytes, v_dst, seg_bytes)))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_out overlaps the cache rows being written");
+  a.q_in = static_cast<const uint16_t *>(q_in);
+  a.q_out = static_cast<uint16_t *>(q_out);
+  a.k_in = static_cast<const uint16_t *>(k_seg);
+  a.k_out = k_dst;
+  a.v_in = static_cast<const uint16_t *>(v_seg);
+  a.v_out = v_dst;
+  a.n_q_rows = q_rows;
+  a.n_kv_rows = n_tokens;
+  a.n_video = cfg != nullptr ? n_tokens : 0;
+  if (layout != nullptr) {
+    a.grid_h = layout->grid_h;
+    a.grid_w = layout->grid_w;
+    a.t0 = layout->t0;
+  }
+  if (q_rows > 0 || n_tokens > 0) {
+    const cudaError_t e = launch_rope_append(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  cache->len += n_tokens;
+  return ok();
+}
+
+nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame_idx,
+                                  int32_t n_frames, int32_t idx_on_device, nomas_kvcache *window,
+                                  int32_t *dev_err, void *stream) {
+  if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
+  nomas_status st = check_shape(src->heads, src->head_dim);
+  if (st != NOMAS_OK) return st;
+  if ((st = check_shape(window->heads, window->head_dim)) != NOMAS_OK) return st;
+  if (src->tokens_per_frame <= 0) return fail(NOMAS_ERR_INVALID_ARG, "src tokens_per_frame <= 0");
+  if (n_frames < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_frames < 0");
+  if (src->len < 0 || src->len > src->capacity || window->capacity < 0)
+    return fail(NOMAS_ERR_INVALID_ARG, "src len/capacity inconsistent");
+  const int64_t P = src->tokens_per_frame;
+  const int64_t rows = (int64_t)n_frames * P;
+  if (rows > window->capacity)
+    return fail(NOMAS_ERR_CAPACITY, "window capacity %lld < %d frames x %lld rows",
+                (long long)window->capacity, n_frames, (long long)P);
+  if (n_frames > 0) {
+    if (frame_idx == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "frame_idx is NULL");
+    if (src->k == nullptr || src->v == nullptr || window->k == nullptr || window->v == nullptr ||
+        !aligned16(src->k) || !aligned16(src->v) || !aligned16(window->k) || !aligned16(window->v))
+      return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
+    const int64_t sb = src->len * kRowBytes, wb = rows * kRowBytes;
+    if (overlap(src->k, sb, window->k, wb) || overlap(src->v, sb, window->v, wb) ||
+        overlap(src->k, sb, window->v, wb) || overlap(src->v, sb, window->k, wb) ||
+        overlap(window->k, wb, window->v, wb))
+      return fail(NOMAS_ERR_INVALID_ARG, "window overlaps the source cache");
+  }
+  const int64_t n_src_frames = src->len / P;
+  if (idx_on_device && n_frames > 0 && dev_err == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "dev_err is required for a device-resident frame list");
+  if (!idx_on_device) {
+    for (int32_t j = 0; j < n_frames; ++j)
+      if (frame_idx[j] < 0 || frame_idx[j] >= n_src_frames)
+        return fail(NOMAS_ERR_INDEX, "frame_idx[%d] = %d outside [0, %lld)", j, frame_idx[j],
+                    (long long)n_src_frames);
+  }
+  SelectArgs a{};
+  a.src_k = static_cast<const uint16_t *>(src->k);
+  a.src_v = static_cast<const uint16_t *>(src->v);
+  a.dst_k = static_cast<uint16_t *>(window->k);
+  a.dst_v = static_cast<uint16_t *>(window->v);
+  a.dev_err = dev_err;
+  a.frame_vecs = P * kRowVecs;
+  a.n_src_frames = n_src_frames;
+  const int chunk = idx_on_device ? 65535 : kSelectHostFramesPerLaunch;
+  SelectHostList hl;
+  for (int32_t f0 = 0; f0 < n_frames; f0 += chunk) {
+    const int32_t nf = (n_frames - f0) < chunk ? (n_frames - f0) : chunk;
+    a.first_frame = f0;
+    a.n_frames = nf;
+    if (idx_on_device) {
+      a.idx_dev = frame_idx;
+    } else {
+      a.idx_dev = nullptr;
+      std::memcpy(hl.idx, frame_idx + f0, sizeof(int32_t) * nf);
+    }
+    const cudaError_t e =
+        launch_select(a, idx_on_device ? nullptr : &hl, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  }
+  window->tokens_per_frame = src->tokens_per_frame;
+  window->len = rows;
+  return ok();
+}
+
+nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                     int32_t n_spans, void *o, float *lse, float softmax_scale,
+                                     int32_t heads, int32_t head_dim, int32_t *dev_err,
+                                     void *stream) {
+  nomas_status st = check_shape(heads, head_dim);
+  if (st != NOMAS_OK) return st;
+  if (n_spans < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_spans < 0");
+  if (n_spans > kMaxSpans)
+    return fail(NOMAS_ERR_UNSUPPORTED, "at most %d key/value spans (got %d)", kMaxSpans, n_spans);
+  if (n_spans > 0 && spans == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "spans is NULL");
+  if (n_q < 0 || n_q > 0x7fff0000LL) return fail(NOMAS_ERR_INVALID_ARG, "n_q out of range");
+  if (n_q == 0) return ok();
+  if (q == nullptr || o == nullptr || !aligned16(q) || !aligned16(o))
+    return fail(NOMAS_ERR_INVALID_ARG, "q and o must be non-NULL and 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return fail(NOMAS_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(NOMAS_ERR_INVALID_ARG, "softmax_scale not finite");
+  const int64_t qb = n_q * kRowBytes;
+  if (overlap(q, qb, o, qb)) return fail(NOMAS_ERR_INVALID_ARG, "o overlaps q");
+  if (lse != nullptr && (overlap(lse, n_q * kHeads * 4, o, qb) || overlap(lse, n_q * kHeads * 4, q, qb)))
+    return fail(NOMAS_ERR_INVALID_ARG, "lse overlaps q or o");
+  AttnArgs a{};
+  int n_used = 0;
+  for (int s = 0; s < n_spans; ++s) {
+    const nomas_kv_span &sp = spans[s];
+    if (sp.len < 0 || sp.len > 0x7fff0000LL)
+      return fail(NOMAS_ERR_INVALID_ARG, "span %d length out of range", s);
+    if (sp.len == 0) continue;
+    if (sp.k == nullptr || sp.v == nullptr || !aligned16(sp.k) || !aligned16(sp.v))
+      return fail(NOMAS_ERR_INVALID_ARG, "span %d k/v must be non-NULL and 16-byte aligned", s);
+    const int64_t sbytes = sp.len * kRowBytes;
+    if (overlap(sp.k, sbytes, o, qb) || overlap(sp.v, sbytes, o, qb) ||
+        (lse != nullptr && (overlap(sp.k, sbytes, lse, n_q * kHeads * 4) ||
+                            overlap(sp.v, sbytes, lse, n_q * kHeads * 4))))
+      return fail(NOMAS_ERR_INVALID_ARG, "span %d overlaps an output", s);
+    if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len)) != NOMAS_OK) return st;
+    if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len)) != NOMAS_OK) return st;
+    a.span_len[n_used] = sp.len;
+    ++n_used;
+  }
+  if (n_used == 0) {
+    const cudaError_t e = launch_attention_empty(static_cast<uint16_t *>(o), lse, n_q,
+                                                 static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention (no keys) launch");
+    return ok();
+  }
+  if ((st = rows_map(&a.tmap_q, q, n_q)) != NOMAS_OK) return st;
+  const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)kHeadDim);
+  a.scale_log2 = (float)(scale * 1.4426950408889634);
+  a.n_spans = n_used;
+  a.n_q = (int32_t)n_q;
+  a.o = static_cast<uint16_t *>(o);
+  a.lse = lse;
+  a.dev_err = dev_err;
+  a.wait_limit_ns = g_wait_limit_ns;
+  const cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,551 @@
+// Segment-over-cache attention for sm_100a: TMA -> shared memory ->
+// tcgen05.mma with TMEM accumulators, fp32 online softmax, no mask.
+//
+// "Hy-Nomas: an 8.6B world model whose memory is a KV cache"
+// (ai.thesatyajit.com), section "How one segment is made" (joint attention of
+// text and video tokens, 16 heads of 128, causal across segments: the current
+// segment reads earlier ones from the KV cache and sees itself and the text
+// in full) and section "What 'world memory' stores" (the queries of segment k
+// attend over the cached keys and values).
+//
+// Work unit: one CTA = one head x 256 query rows, as two 128-row Q tiles that
+// share every K/V tile.  Keys stream through a ring of 32-KiB shared-memory
+// slots, K and V tiles alternating, 128 keys per tile, across up to four
+// spans (cache or window, text, segment), each with its own tensor map; TMA
+// zero-fills rows past a span's end and the softmax masks them.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for Q tile 0 (TMEM lanes 0-127, one query row per thread)
+//   warps 4-7  softmax for Q tile 1
+//   warp 8     TMA producer (one elected lane)
+//   warp 9     MMA issuer (one elected lane); owns the TMEM allocation
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
+// P_i (bf16, 64 columns) overwrites the first half of S_i once the softmax has
+// read S_i into registers, and is the TMEM A operand of O_i += P_i V.
+//
+// Issue order of the MMA lane, per K/V tile j:
+//   O0 += P0(j) V_j ; S0 = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1 = Q1 K_{j+1}^T
+// so each softmax group works on one tile while the tensor core runs the
+// other tile's two GEMMs.  tcgen05 operations of one thread complete in issue
+// order, so the commit that announces S_i(j+1) also covers O_i += P_i(j) V_j:
+// when a softmax thread sees S_i ready, O_i is quiescent and the thread may
+// rescale it in place.  Rescaling is lazy: the running max is only raised
+// when a row's new max exceeds it by more than 2^8 (log2 domain), otherwise P
+// is formed against the stale max (values up to 256) and the final division
+// by the row sum, formed with the same max, makes the result exact.
+//
+// Every wait is bounded (a globaltimer limit); on expiry the kernel records
+// NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and
+// returns.
+#include <cuda_bf16.h>
+
+#include "nomas_internal.h"
+#include "tmem_ops.cuh"
+
+namespace nomas {
+namespace {
+
+constexpr int kBM = 128;              // query rows per Q tile (MMA M)
+constexpr int kBN = 128;              // keys per K/V tile (MMA N of QK^T)
+constexpr int kQTiles = 2;
+constexpr int kStages = 4;            // K/V ring slots
+constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KiB
+constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+
+// Shared-memory map (offsets from a 1024-B aligned base).
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = kOffQ + kQTiles * kTileBytes;
+constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
+// barrier indices (8 B each)
+constexpr int kBarQFull = 0;
+constexpr int kBarKVFull = 1;                      // + slot
+constexpr int kBarKVEmpty = kBarKVFull + kStages;  // + slot
+constexpr int kBarSFull = kBarKVEmpty + kStages;   // + tile
+constexpr int kBarPFull = kBarSFull + 2;           // + tile
+constexpr int kBarOFull = kBarPFull + 2;           // + tile
+constexpr int kBarDrain = kBarOFull + 2;
+constexpr int kNumBars = kBarDrain + 1;
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kSmemUsed = kOffAbort + 4;
+constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D,
+// M = 128, N = 128; A K-major; B K-major (QK^T: K rows are key-major with
+// dims contiguous) or MN-major (PV: V rows have dims, i.e. N, contiguous).
+constexpr uint32_t make_idesc(uint32_t b_mn_major) {
+  return (1u << 4)            // D format f32
+       | (1u << 7)            // A format bf16
+       | (1u << 10)           // B format bf16
+       | (b_mn_major << 16)   // B major
+       | ((128u >> 3) << 17)  // N
+       | ((128u >> 4) << 24); // M
+}
+constexpr uint32_t kIdescQK = make_idesc(0);
+constexpr uint32_t kIdescPV = make_idesc(1);
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// ---------------------------------------------------------------- mbarrier --
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+struct WaitCtl {
+  volatile int *abort;              // CTA-wide abort flag in shared memory
+  int32_t *dev_err;
+  unsigned long long limit_ns;
+};
+
+// Slow path of wait_phase: spins until the phase completes, the CTA aborts,
+// or the time limit passes (then it raises the abort flag and reports).
+__device__ __forceinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, volatile int *abort,
+                                             int32_t *dev_err, unsigned long long limit_ns) {
+  const unsigned long long start = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - start > limit_ns) {
+        *abort = 1;
+        if (dev_err != nullptr) atomicOr(dev_err, NOMAS_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Waits for the phase of `bar` with the given parity.  Returns false when the
+// CTA is aborting (this wait ran out of time, or another role's did).
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtl &c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, c.abort, c.dev_err, c.limit_ns);
+}
+
+// Teardown wait for operations this thread started itself: ignores the abort
+// flag, still bounded.
+__device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long start = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - start > limit_ns) return;
+  }
+}
+
+// --------------------------------------------------------------------- TMA --
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05 --
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// S = Q_i K^T over D = 128: 8 MMAs of K = 16.  Both operands K-major, 128-B
+// swizzled, two 16-KiB halves (dims 0-63, 64-127); a K step of 16 elements
+// advances the start address by 32 B inside a swizzle atom.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t off = (uint32_t)(k >> 2) * kHalfBytes + (uint32_t)(k & 3) * 32u;
+    mma_ss(d_tmem, sw128_desc(q_smem + off, 16, 1024), sw128_desc(k_smem + off, 16, 1024),
+           kIdescQK, k > 0 ? 1u : 0u);
+  }
+}
+
+// O_i (+)= P_i V over 128 keys: 8 MMAs of K = 16 keys.  P comes from TMEM
+// (8 columns of packed bf16 pairs per step); V is MN-major: 8-key groups are
+// 1024 B apart (SBO), the two 64-dim halves 16 KiB apart (LBO).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
+                                         bool accumulate) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    mma_ts(d_tmem, p_tmem + (uint32_t)k * 8u, sw128_desc(v_smem + (uint32_t)k * 2048u, kHalfBytes, 1024),
+           kIdescPV, (accumulate || k > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ int num_tiles(int64_t len) { return (int)((len + kBN - 1) / kBN); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+attention_kernel(const __grid_constant__ AttnArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *const gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int head = blockIdx.y;
+  const int q_row0 = blockIdx.x * (kQTiles * kBM);
+
+  const uint32_t sQ = base + kOffQ;
+  const uint32_t sKV = base + kOffKV;
+  auto bar = [&](int i) { return base + kOffBar + (uint32_t)i * 8u; };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + kOffTmemSlot);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQFull), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarKVFull + s), 1);
+      mbar_init(bar(kBarKVEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(kBarSFull + t), 1);
+      mbar_init(bar(kBarPFull + t), 128);
+      mbar_init(bar(kBarOFull + t), 1);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const WaitCtl ctl{abort_flag, p.dev_err, p.wait_limit_ns};
+  int n_kv = 0;
+  for (int s = 0; s < p.n_spans; ++s) n_kv += num_tiles(p.span_len[s]);
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(bar(kBarQFull), kQTiles * kTileBytes);
+      for (int i = 0; i < kQTiles; ++i)
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sQ + i * kTileBytes + c * kHalfBytes, &p.tmap_q, bar(kBarQFull),
+                      head * kHeadDim + c * 64, q_row0 + i * kBM);
+      int t = 0;
+      bool ok = true;
+      for (int s = 0; s < p.n_spans && ok; ++s) {
+        const int nt = num_tiles(p.span_len[s]);
+        for (int kt = 0; kt < nt && ok; ++kt) {
+          for (int which = 0; which < 2; ++which, ++t) {
+            const int slot = t % kStages;
+            const uint32_t ph = (uint32_t)(t / kStages) & 1u;
+            if (!wait_phase(bar(kBarKVEmpty + slot), ph ^ 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(bar(kBarKVFull + slot), kTileBytes);
+            const CUtensorMap *m = which == 0 ? &p.tmap_k[s] : &p.tmap_v[s];
+            for (int c = 0; c < 2; ++c)
+              tma_load_2d(sKV + slot * kTileBytes + c * kHalfBytes, m, bar(kBarKVFull + slot),
+                          head * kHeadDim + c * 64, kt * kBN);
+          }
+        }
+      }
+      // Teardown: wait until every load this lane issued has landed.
+      drain_phase(bar(kBarQFull), 0, p.wait_limit_ns);
+      for (int u = (t > kStages ? t - kStages : 0); u < t; ++u)
+        drain_phase(bar(kBarKVFull + u % kStages), (uint32_t)(u / kStages) & 1u, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0 && n_kv > 0) {
+      const uint32_t tS[2] = {tmem_base + 0u, tmem_base + 128u};
+      const uint32_t tO[2] = {tmem_base + 256u, tmem_base + 384u};
+      auto slot_of = [](int t) { return t % kStages; };
+      auto ph_of = [](int t) { return (uint32_t)(t / kStages) & 1u; };
+      do {
+        if (!wait_phase(bar(kBarQFull), 0, ctl)) break;
+        if (!wait_phase(bar(kBarKVFull + slot_of(0)), ph_of(0), ctl)) break;
+        tc_fence_after();
+        const uint32_t k0 = sKV + slot_of(0) * kTileBytes;
+        issue_qk(tS[0], sQ, k0);
+        mma_commit(bar(kBarSFull + 0));
+        issue_qk(tS[1], sQ + kTileBytes, k0);
+        mma_commit(bar(kBarSFull + 1));
+        mma_commit(bar(kBarKVEmpty + slot_of(0)));
+        for (int j = 0; j < n_kv; ++j) {
+          const int tv = 2 * j + 1, tk = 2 * j + 2;
+          const uint32_t vs = sKV + slot_of(tv) * kTileBytes;
+          const uint32_t ks = sKV + slot_of(tk) * kTileBytes;
+          const uint32_t par = (uint32_t)j & 1u;
+          const bool more = j + 1 < n_kv;
+          if (!wait_phase(bar(kBarKVFull + slot_of(tv)), ph_of(tv), ctl)) break;
+          if (!wait_phase(bar(kBarPFull + 0), par, ctl)) break;
+          tc_fence_after();
+          issue_pv(tO[0], tS[0], vs, j > 0);
+          if (more) {
+            if (!wait_phase(bar(kBarKVFull + slot_of(tk)), ph_of(tk), ctl)) break;
+            tc_fence_after();
+            issue_qk(tS[0], sQ, ks);
+            mma_commit(bar(kBarSFull + 0));
+          } else {
+            mma_commit(bar(kBarOFull + 0));
+          }
+          if (!wait_phase(bar(kBarPFull + 1), par, ctl)) break;
+          tc_fence_after();
+          issue_pv(tO[1], tS[1], vs, j > 0);
+          mma_commit(bar(kBarKVEmpty + slot_of(tv)));
+          if (more) {
+            issue_qk(tS[1], sQ + kTileBytes, ks);
+            mma_commit(bar(kBarSFull + 1));
+            mma_commit(bar(kBarKVEmpty + slot_of(tk)));
+          } else {
+            mma_commit(bar(kBarOFull + 1));
+          }
+        }
+      } while (false);
+      // Teardown: every MMA issued above completes before TMEM is freed.
+      mma_commit(bar(kBarDrain));
+      drain_phase(bar(kBarDrain), 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int tile = warp >> 2;
+    const int quarter = warp & 3;
+    const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem_base + lane_bits + (uint32_t)tile * 128u;
+    const uint32_t tO = tmem_base + lane_bits + 256u + (uint32_t)tile * 128u;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale)
+    float l = 0.f;        // running row sum of exp2(...)
+    bool ok = true;
+    int j = 0;
+    for (int s = 0; s < p.n_spans && ok; ++s) {
+      const int64_t len = p.span_len[s];
+      const int nt = num_tiles(len);
+      for (int kt = 0; kt < nt; ++kt, ++j) {
+        if (!wait_phase(bar(kBarSFull + tile), (uint32_t)j & 1u, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem::ld32(tS + 0, sr + 0);
+        tmem::ld32(tS + 32, sr + 32);
+        tmem::ld32(tS + 64, sr + 64);
+        tmem::ld32(tS + 96, sr + 96);
+        tmem::wait_ld128(sr);
+        float *sv = reinterpret_cast<float *>(sr);
+        const int64_t rem = len - (int64_t)kt * kBN;
+        if (rem < kBN) {
+          const int valid = (int)rem;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) sv[c] = -INFINITY;
+        }
+        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          m0 = fmaxf(m0, sv[c]);
+          m1 = fmaxf(m1, sv[c + 1]);
+          m2 = fmaxf(m2, sv[c + 2]);
+          m3 = fmaxf(m3, sv[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+        // Lazy max: raise it (and rescale O and l by alpha) only when some
+        // row of the warp grew by more than 2^8; the O update happens after
+        // P is stored, while the S values are no longer live.
+        bool rescale = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m = mx;
+        } else if (__any_sync(0xffffffffu, mx > m + 8.0f)) {
+          const float m_new = fmaxf(m, mx);
+          alpha = ex2(m - m_new);
+          m = m_new;
+          l *= alpha;
+          rescale = true;
+        }
+        const float neg_m = -m;
+        float l0 = 0.f, l1 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float e0 = ex2(fmaf(sv[2 * c], sl2, neg_m));
+          const float e1 = ex2(fmaf(sv[2 * c + 1], sl2, neg_m));
+          l0 += e0;
+          l1 += e1;
+          pk[c] = pack_bf16x2(e0, e1);
+        }
+        l += l0 + l1;
+        tmem::st32(tS + 0, pk);
+        tmem::st32(tS + 32, pk + 32);
+        if (rescale) {
+#pragma unroll
+          for (int cc = 0; cc < 128; cc += 32) {
+            uint32_t orow[32];
+            tmem::ld32(tO + cc, orow);
+            tmem::wait_ld32(orow);
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha);
+            tmem::st32(tO + cc, orow);
+          }
+        }
+        tmem::wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + tile));
+      }
+    }
+    // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l).
+    if (ok && n_kv > 0 && wait_phase(bar(kBarOFull + tile), 0, ctl)) {
+      tc_fence_after();
+      const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
+      const float inv_l = 1.0f / l;
+      uint16_t *orow_g = p.o + row * kRowElems + head * kHeadDim;
+#pragma unroll
+      for (int cc = 0; cc < 128; cc += 32) {
+        uint32_t orow[32];
+        tmem::ld32(tO + cc, orow);
+        tmem::wait_ld32(orow);
+        if (row < p.n_q) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow_g + cc);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(orow[8 * v + 0]) * inv_l, __uint_as_float(orow[8 * v + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(orow[8 * v + 2]) * inv_l, __uint_as_float(orow[8 * v + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(orow[8 * v + 4]) * inv_l, __uint_as_float(orow[8 * v + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(orow[8 * v + 6]) * inv_l, __uint_as_float(orow[8 * v + 7]) * inv_l);
+            dst[v] = w;
+          }
+        }
+      }
+      if (p.lse != nullptr && row < p.n_q)
+        p.lse[(int64_t)head * p.n_q + row] = (m + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// Zero keys: O = 0, LSE = -inf.
+__global__ void attention_empty_kernel(uint16_t *o, float *lse, int64_t n_q) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t n_vec = n_q * kRowVecs;
+  for (int64_t v = i; v < n_vec; v += (int64_t)gridDim.x * blockDim.x)
+    reinterpret_cast<uint4 *>(o)[v] = make_uint4(0, 0, 0, 0);
+  if (lse != nullptr)
+    for (int64_t v = i; v < n_q * kHeads; v += (int64_t)gridDim.x * blockDim.x) lse[v] = -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
+  // The shared-memory opt-in is a per-device function attribute.
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t q_blocks = ((int64_t)a.n_q + kQTiles * kBM - 1) / (kQTiles * kBM);
+  if (q_blocks <= 0) return cudaSuccess;
+  if (q_blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)q_blocks, kHeads);
+  attention_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q, cudaStream_t stream) {
+  if (n_q <= 0) return cudaSuccess;
+  attention_empty_kernel<<<1184, 256, 0, stream>>>(o, lse, n_q);
+  return cudaGetLastError();
+}
+
+}  // namespace nomas

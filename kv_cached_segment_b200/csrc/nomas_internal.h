@@ -1,0 +1,74 @@
+// Internal interfaces between the C-ABI layer (abi.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nomas.h"
+
+namespace nomas {
+
+constexpr int kHeads = 16;
+constexpr int kHeadDim = 128;
+constexpr int kRowElems = kHeads * kHeadDim;       // 2048 bf16
+constexpr int64_t kRowBytes = kRowElems * 2;       // 4096 B
+constexpr int kRowVecs = kRowBytes / 16;           // 256 x 16 B
+
+// ---------------------------------------------------------------- RoPE ----
+struct RopeArgs {
+  const uint16_t *q_in;   // may be null
+  uint16_t *q_out;
+  const uint16_t *k_in;   // may be null
+  uint16_t *k_out;
+  const uint16_t *v_in;   // may be null (no V stream)
+  uint16_t *v_out;
+  int64_t n_q_rows;       // rows of Q processed (video + text)
+  int64_t n_kv_rows;      // rows of K (and V) processed
+  int64_t n_video;        // rows [0, n_video) are rotated (0: plain copy)
+  int32_t grid_h, grid_w, t0;
+  // Per-pair angular frequency (radians per position unit) and the axis
+  // (0 = t, 1 = h, 2 = w) of the 64 rotation pairs of a head.
+  double omega[kHeadDim / 2];
+  int8_t axis[kHeadDim / 2];
+};
+cudaError_t launch_rope_append(const RopeArgs &a, cudaStream_t stream);
+
+// -------------------------------------------------------------- select ----
+constexpr int kSelectHostFramesPerLaunch = 2048;
+struct SelectArgs {
+  const uint16_t *src_k, *src_v;
+  uint16_t *dst_k, *dst_v;
+  const int32_t *idx_dev;      // device list, or null for the host list below
+  int32_t *dev_err;
+  int64_t frame_vecs;          // 16-B vectors per frame per tensor
+  int64_t n_src_frames;
+  int32_t n_frames;            // frames handled by this launch
+  int32_t first_frame;         // window frame of entry 0 of this launch
+};
+struct SelectHostList {
+  int32_t idx[kSelectHostFramesPerLaunch];
+};
+cudaError_t launch_select(const SelectArgs &a, const SelectHostList *host_list,
+                          cudaStream_t stream);
+
+// ----------------------------------------------------------- attention ----
+constexpr int kMaxSpans = 4;
+struct AttnArgs {
+  CUtensorMap tmap_q;
+  CUtensorMap tmap_k[kMaxSpans];
+  CUtensorMap tmap_v[kMaxSpans];
+  int64_t span_len[kMaxSpans];
+  int32_t n_spans;             // non-empty spans, packed to the front
+  int32_t n_q;
+  uint16_t *o;
+  float *lse;                  // may be null
+  float scale_log2;            // softmax scale * log2(e)
+  int32_t *dev_err;            // may be null
+  unsigned long long wait_limit_ns;
+};
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
+cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
+                                   cudaStream_t stream);
+
+}  // namespace nomas

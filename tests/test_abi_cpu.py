@@ -1,0 +1,201 @@
+"""C-ABI checks that need no GPU.
+
+The library must load on a machine without a GPU driver, export every symbol
+include/nomas.h declares, and reject bad arguments on the host, before any
+launch, with the documented status codes.  The fake device pointers used here
+are never dereferenced: every call below fails validation first.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kv_cached_segment_b200 as nm
+from kv_cached_segment_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+ROW = 4096
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return nm.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "nomas.h")).read()
+    return sorted(set(re.findall(r"\b(nomas_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert set(nm.EXPORTED_SYMBOLS) <= set(names) | {"nomas_last_error", "nomas_version"}
+    for name in names:
+        assert hasattr(lib, name), name
+    # and the dynamic symbol table really carries them
+    out = os.popen(f"nm -D --defined-only {nm.library_path()}").read()
+    for name in names:
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_version_and_empty_error(lib):
+    assert b"sm_100a" in lib.nomas_version()
+    assert lib.nomas_last_error() is not None
+
+
+def _layout(frames=2, gh=4, gw=6, t0=2, n_text=64):
+    return nm._SegLayout(frames, gh, gw, t0, n_text)
+
+
+def _cfg(dt=32, dh=48, dw=48, theta=10000.0):
+    return nm._RopeCfg(dt, dh, dw, theta)
+
+
+def test_rope_rejects_unsupported_heads(lib):
+    st = lib.nomas_rope3d_qk(FAKE, FAKE, FAKE + ROW * 1000, FAKE + ROW * 2000,
+                             ctypes.byref(_layout()), ctypes.byref(_cfg()), 8, 128, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED
+    assert b"heads" in lib.nomas_last_error()
+    st = lib.nomas_rope3d_qk(FAKE, None, FAKE, None, ctypes.byref(_layout()),
+                             ctypes.byref(_cfg()), 16, 64, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("cfg", [_cfg(32, 48, 40), _cfg(31, 49, 48), _cfg(0, 64, 64),
+                                 _cfg(32, 48, 48, 0.0), _cfg(32, 48, 48, float("inf"))])
+def test_rope_rejects_bad_config(lib, cfg):
+    st = lib.nomas_rope3d_qk(FAKE, None, FAKE, None, ctypes.byref(_layout()), ctypes.byref(cfg),
+                             16, 128, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+
+
+def test_rope_rejects_misaligned_and_null(lib):
+    st = lib.nomas_rope3d_qk(FAKE + 8, None, FAKE + 8, None, ctypes.byref(_layout()),
+                             ctypes.byref(_cfg()), 16, 128, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    st = lib.nomas_rope3d_qk(None, None, FAKE, None, ctypes.byref(_layout()),
+                             ctypes.byref(_cfg()), 16, 128, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    st = lib.nomas_rope3d_qk(FAKE, FAKE, FAKE, None, ctypes.byref(_layout()),
+                             ctypes.byref(_cfg()), 16, 128, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    bad = _layout(frames=-1)
+    st = lib.nomas_rope3d_qk(FAKE, None, FAKE, None, ctypes.byref(bad), ctypes.byref(_cfg()),
+                             16, 128, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+
+
+def _cache(capacity, length, tpf=24, heads=16, head_dim=128, base=FAKE):
+    return nm._KVCache(base, base + capacity * ROW, capacity, length, tpf, heads, head_dim)
+
+
+def test_append_capacity_overflow_leaves_len(lib):
+    c = _cache(100, 60)
+    seg = FAKE + 10 ** 9
+    st = lib.nomas_kvcache_append(ctypes.byref(c), seg, seg + 48 * ROW, 48, None, None,
+                                  ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_CAPACITY and c.len == 60
+    assert b"capacity" in lib.nomas_last_error()
+
+
+def test_append_validation(lib):
+    seg = FAKE + 10 ** 9
+    c = _cache(1000, 0)
+    # n_tokens must match the layout's video rows when rotating
+    st = lib.nomas_kvcache_append(ctypes.byref(c), seg, seg + 48 * ROW, 47, None, None,
+                                  ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    # a rope config needs a layout
+    st = lib.nomas_kvcache_append(ctypes.byref(c), seg, seg + 48 * ROW, 48, None, None, None,
+                                  ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    # q_in without q_out
+    st = lib.nomas_kvcache_append(ctypes.byref(c), seg, seg + 48 * ROW, 48, seg + 96 * ROW, None,
+                                  ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    # segment overlapping the rows being written
+    st = lib.nomas_kvcache_append(ctypes.byref(c), FAKE, seg, 48, None, None,
+                                  ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    # unsupported cache geometry
+    c2 = _cache(1000, 0, heads=8)
+    st = lib.nomas_kvcache_append(ctypes.byref(c2), seg, seg + 48 * ROW, 48, None, None, None,
+                                  None, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED
+    # len beyond capacity is inconsistent
+    c3 = _cache(10, 11)
+    st = lib.nomas_kvcache_append(ctypes.byref(c3), seg, seg + ROW, 0, None, None, None, None,
+                                  None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    assert c.len == 0
+
+
+def test_append_of_nothing_is_ok_without_launch(lib):
+    c = _cache(10, 4)
+    st = lib.nomas_kvcache_append(ctypes.byref(c), None, None, 0, None, None, None, None, None)
+    assert st == nm.NOMAS_OK and c.len == 4
+
+
+def test_select_validation(lib):
+    src = _cache(240, 240, tpf=24)
+    win = _cache(96, 0, tpf=0, base=FAKE + 10 ** 9)
+    idx = (ctypes.c_int32 * 4)(0, 3, 10, 2)  # 240 rows / 24 = 10 frames
+    st = lib.nomas_kvcache_select(ctypes.byref(src), idx, 4, 0, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_INDEX and win.len == 0
+    assert b"frame_idx[2]" in lib.nomas_last_error()
+    neg = (ctypes.c_int32 * 1)(-1)
+    st = lib.nomas_kvcache_select(ctypes.byref(src), neg, 1, 0, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_INDEX
+    idx5 = (ctypes.c_int32 * 5)(0, 1, 2, 3, 4)  # 5 x 24 rows > 96
+    st = lib.nomas_kvcache_select(ctypes.byref(src), idx5, 5, 0, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_CAPACITY
+    st = lib.nomas_kvcache_select(ctypes.byref(src), FAKE, 2, 1, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG and b"dev_err" in lib.nomas_last_error()
+    overl = _cache(96, 0, tpf=0, base=FAKE + 10 * ROW)
+    ok_idx = (ctypes.c_int32 * 2)(0, 1)
+    st = lib.nomas_kvcache_select(ctypes.byref(src), ok_idx, 2, 0, ctypes.byref(overl), None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    src0 = _cache(240, 240, tpf=0)
+    st = lib.nomas_kvcache_select(ctypes.byref(src0), ok_idx, 2, 0, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+
+
+def test_attention_validation(lib):
+    spans = (nm._KVSpan * 5)(*[nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, 10)] * 5)
+    o = FAKE + 3 * 10 ** 9
+    st = lib.nomas_segment_attention(FAKE, 100, spans, 5, o, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED
+    st = lib.nomas_segment_attention(FAKE, 100, spans, 1, o, None, 0.0, 16, 96, None, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED
+    st = lib.nomas_segment_attention(FAKE, 100, spans, 1, FAKE + 16, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG  # o overlaps q
+    st = lib.nomas_segment_attention(FAKE + 4, 100, spans, 1, o, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG  # misaligned
+    st = lib.nomas_segment_attention(FAKE, 100, spans, 1, o, None, float("nan"), 16, 128, None,
+                                     None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    bad = (nm._KVSpan * 1)(nm._KVSpan(None, None, 10))
+    st = lib.nomas_segment_attention(FAKE, 100, bad, 1, o, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    neg = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, -1))
+    st = lib.nomas_segment_attention(FAKE, 100, neg, 1, o, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    over = (nm._KVSpan * 1)(nm._KVSpan(o, FAKE + 2 * 10 ** 9, 10))
+    st = lib.nomas_segment_attention(FAKE, 100, over, 1, o, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG  # a span overlaps the output
+    # no query rows: nothing to do, nothing launched
+    st = lib.nomas_segment_attention(None, 0, spans, 1, None, None, 0.0, 16, 128, None, None)
+    assert st == nm.NOMAS_OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = nm._lib
+    try:
+        nm._lib = None
+        with pytest.raises(ImportError):
+            nm.load_library(str(tmp_path / "missing.so"))
+    finally:
+        nm._lib = saved
