@@ -39,7 +39,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=40)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["nomas", "reference"], default="nomas")
-    p.add_argument("--workload", choices=["720p", "bounded", "mid", "tiny"], default="720p")
+    p.add_argument("--workload", choices=["720p", "bounded", "short", "mid", "tiny"], default="720p")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()

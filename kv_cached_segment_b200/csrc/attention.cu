@@ -26,7 +26,8 @@
 // Issue order of the MMA lane, per K/V tile j:
 //   O0 += P0(j) V_j ; S0 = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1 = Q1 K_{j+1}^T
 // so each softmax group works on one tile while the tensor core runs the
-// other tile's two GEMMs.  tcgen05 operations of one thread complete in issue
+// other tile's two GEMMs.  P is published in two halves of 64 keys, so the
+// first half of O += P V runs while the softmax computes the second half.  tcgen05 operations of one thread complete in issue
 // order, so the commit that announces S_i(j+1) also covers O_i += P_i(j) V_j:
 // when a softmax thread sees S_i ready, O_i is quiescent and the thread may
 // rescale it in place.  Rescaling is lazy: the running max is only raised
@@ -48,7 +49,10 @@ namespace {
 constexpr int kBM = 128;              // query rows per Q tile (MMA M)
 constexpr int kBN = 128;              // keys per K/V tile (MMA N of QK^T)
 constexpr int kQTiles = 2;
-constexpr int kStages = 4;            // K/V ring slots
+#ifndef NOMAS_ATTN_STAGES
+#define NOMAS_ATTN_STAGES 5
+#endif
+constexpr int kStages = NOMAS_ATTN_STAGES;  // K/V ring slots
 constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KiB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
 constexpr int kProducerWarp = 8;
@@ -66,7 +70,8 @@ constexpr int kBarKVFull = 1;                      // + slot
 constexpr int kBarKVEmpty = kBarKVFull + kStages;  // + slot
 constexpr int kBarSFull = kBarKVEmpty + kStages;   // + tile
 constexpr int kBarPFull = kBarSFull + 2;           // + tile
-constexpr int kBarOFull = kBarPFull + 2;           // + tile
+constexpr int kBarPHalf = kBarPFull + 2;           // + tile: first 64 keys of P
+constexpr int kBarOFull = kBarPHalf + 2;           // + tile
 constexpr int kBarDrain = kBarOFull + 2;
 constexpr int kNumBars = kBarDrain + 1;
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
@@ -168,13 +173,26 @@ __device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity, unsig
 }
 
 // --------------------------------------------------------------------- TMA --
+// 2-D tiled TMA load into shared memory, completing on `bar`, with an L2
+// eviction-priority policy (K/V tiles are re-read by every query block of the
+// head and should stay in L2; Q is read once).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int32_t x, int32_t y) {
+                                            int32_t x, int32_t y, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 // ----------------------------------------------------------------- tcgen05 --
@@ -184,13 +202,17 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// One tcgen05.mma kind::f16 with both operands in shared memory (SS) or A in
+// tensor memory (TS).  ACC = 0 overwrites D, 1 accumulates into it; the
+// predicate comes from an immediate so the issue costs one instruction.
+template <int ACC>
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+                                       uint32_t idesc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(ACC)
       : "memory");
 }
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -219,28 +241,104 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ---------------------------------------------------- packed fp32 pairs --
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unf2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of values on the FMA pipe, to share the exponential work of
+// the softmax between the MUFU unit and the FMA units.  Cody-Waite style
+// reduction: adding 1.5 * 2^23 rounds x to the nearest integer j (kept in the
+// low mantissa bits of the sum), f = x - j lies in [-1/2, 1/2] exactly, 2^f
+// comes from a degree-3 polynomial whose coefficients were fitted here by the
+// Remez exchange algorithm to minimise the relative error on [-1/2, 1/2]
+// (max 7.5e-5, far below the 2^-9 rounding step of the bf16 P it feeds), and
+// j is added to the exponent field.  x is clamped at -125 so the exponent
+// cannot underflow; 2^-125 stands in for 0.
+constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23
+constexpr float kPc0 = 0.9999280571937561f;
+constexpr float kPc1 = 0.6932609677314758f;
+constexpr float kPc2 = 0.2426111251115799f;
+constexpr float kPc3 = 0.0551716685295105f;
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  float2 v = unf2(x);
+  v.x = fmaxf(v.x, -125.f);
+  v.y = fmaxf(v.y, -125.f);
+  const uint64_t xc = f2(v.x, v.y);
+  const uint64_t t = add2(xc, f2(kShifter, kShifter));
+  const uint64_t jf = add2(t, f2(-kShifter, -kShifter));
+  const uint64_t fr = fma2(jf, f2(-1.f, -1.f), xc);
+  uint64_t pp = fma2(f2(kPc3, kPc3), fr, f2(kPc2, kPc2));
+  pp = fma2(pp, fr, f2(kPc1, kPc1));
+  pp = fma2(pp, fr, f2(kPc0, kPc0));
+  const float2 pv = unf2(pp), tv = unf2(t);
+  return f2(__uint_as_float(__float_as_uint(pv.x) + (__float_as_uint(tv.x) << 23)),
+            __uint_as_float(__float_as_uint(pv.y) + (__float_as_uint(tv.y) << 23)));
+}
+
+// Pairs of P (out of every 8) whose exponentials run on the FMA pipe.
+#ifndef NOMAS_EXP2_FMA_PAIRS
+#define NOMAS_EXP2_FMA_PAIRS 2
+#endif
+__device__ __forceinline__ constexpr bool pair_on_fma(int c) {
+  return (c & 7) < NOMAS_EXP2_FMA_PAIRS;
+}
+
+// The MMA lane must issue an instruction every 64 cycles to keep the tensor
+// core busy (M=128, N=128, K=16 takes 64 cycles), so descriptors are built
+// once and each K step only adds a compile-time offset to the start-address
+// field (bits 0-13, in 16-byte units; addresses stay below 256 KiB, so the
+// add never carries into the other fields).
+__device__ __forceinline__ uint64_t desc_plus(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
 // S = Q_i K^T over D = 128: 8 MMAs of K = 16.  Both operands K-major, 128-B
 // swizzled, two 16-KiB halves (dims 0-63, 64-127); a K step of 16 elements
 // advances the start address by 32 B inside a swizzle atom.
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+  mma_ss<0>(d_tmem, q_desc, k_desc, kIdescQK);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 1; k < 8; ++k) {
     const uint32_t off = (uint32_t)(k >> 2) * kHalfBytes + (uint32_t)(k & 3) * 32u;
-    mma_ss(d_tmem, sw128_desc(q_smem + off, 16, 1024), sw128_desc(k_smem + off, 16, 1024),
-           kIdescQK, k > 0 ? 1u : 0u);
+    mma_ss<1>(d_tmem, desc_plus(q_desc, off), desc_plus(k_desc, off), kIdescQK);
   }
 }
 
-// O_i (+)= P_i V over 128 keys: 8 MMAs of K = 16 keys.  P comes from TMEM
-// (8 columns of packed bf16 pairs per step); V is MN-major: 8-key groups are
-// 1024 B apart (SBO), the two 64-dim halves 16 KiB apart (LBO).
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate) {
+// O_i (+)= P_i V over 64 of the 128 keys of a tile (half 0: keys 0-63, half
+// 1: keys 64-127): 4 MMAs of K = 16 keys.  P comes from TMEM (8 columns of
+// packed bf16 pairs per step); V is MN-major: 8-key groups are 1024 B apart
+// (SBO), the two 64-dim halves 16 KiB apart (LBO); a K step of 16 keys
+// advances the start address by 2 KiB.
+template <int HALF>
+__device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
+                                              uint32_t accumulate) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    mma_ts(d_tmem, p_tmem + (uint32_t)k * 8u, sw128_desc(v_smem + (uint32_t)k * 2048u, kHalfBytes, 1024),
-           kIdescPV, (accumulate || k > 0) ? 1u : 0u);
-  }
+  for (int k = 4 * HALF; k < 4 * HALF + 4; ++k)
+    mma_ts(d_tmem, p_tmem + (uint32_t)k * 8u, desc_plus(v_desc, (uint32_t)k * 2048u), kIdescPV,
+           (k > 0) ? 1u : accumulate);
 }
 
 __device__ __forceinline__ int num_tiles(int64_t len) { return (int)((len + kBN - 1) / kBN); }
@@ -272,6 +370,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(kBarSFull + t), 1);
       mbar_init(bar(kBarPFull + t), 128);
+      mbar_init(bar(kBarPHalf + t), 128);
       mbar_init(bar(kBarOFull + t), 1);
     }
     mbar_init(bar(kBarDrain), 1);
@@ -297,11 +396,13 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
       mbar_expect_tx(bar(kBarQFull), kQTiles * kTileBytes);
       for (int i = 0; i < kQTiles; ++i)
         for (int c = 0; c < 2; ++c)
           tma_load_2d(sQ + i * kTileBytes + c * kHalfBytes, &p.tmap_q, bar(kBarQFull),
-                      head * kHeadDim + c * 64, q_row0 + i * kBM);
+                      head * kHeadDim + c * 64, q_row0 + i * kBM, pol_q);
       int t = 0;
       bool ok = true;
       for (int s = 0; s < p.n_spans && ok; ++s) {
@@ -318,7 +419,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
             const CUtensorMap *m = which == 0 ? &p.tmap_k[s] : &p.tmap_v[s];
             for (int c = 0; c < 2; ++c)
               tma_load_2d(sKV + slot * kTileBytes + c * kHalfBytes, m, bar(kBarKVFull + slot),
-                          head * kHeadDim + c * 64, kt * kBN);
+                          head * kHeadDim + c * 64, kt * kBN, pol_kv);
           }
         }
       }
@@ -335,40 +436,50 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       const uint32_t tO[2] = {tmem_base + 256u, tmem_base + 384u};
       auto slot_of = [](int t) { return t % kStages; };
       auto ph_of = [](int t) { return (uint32_t)(t / kStages) & 1u; };
+      const uint64_t dq0 = sw128_desc(sQ, 16, 1024);
+      const uint64_t dq1 = desc_plus(dq0, kTileBytes);
+      const uint64_t dk = sw128_desc(sKV, 16, 1024);           // slot 0, K-major
+      const uint64_t dv = sw128_desc(sKV, kHalfBytes, 1024);   // slot 0, MN-major
       do {
         if (!wait_phase(bar(kBarQFull), 0, ctl)) break;
         if (!wait_phase(bar(kBarKVFull + slot_of(0)), ph_of(0), ctl)) break;
         tc_fence_after();
-        const uint32_t k0 = sKV + slot_of(0) * kTileBytes;
-        issue_qk(tS[0], sQ, k0);
+        issue_qk(tS[0], dq0, dk);
         mma_commit(bar(kBarSFull + 0));
-        issue_qk(tS[1], sQ + kTileBytes, k0);
+        issue_qk(tS[1], dq1, dk);
         mma_commit(bar(kBarSFull + 1));
         mma_commit(bar(kBarKVEmpty + slot_of(0)));
         for (int j = 0; j < n_kv; ++j) {
           const int tv = 2 * j + 1, tk = 2 * j + 2;
-          const uint32_t vs = sKV + slot_of(tv) * kTileBytes;
-          const uint32_t ks = sKV + slot_of(tk) * kTileBytes;
+          const uint64_t vd = desc_plus(dv, (uint32_t)slot_of(tv) * kTileBytes);
+          const uint64_t kd = desc_plus(dk, (uint32_t)slot_of(tk) * kTileBytes);
           const uint32_t par = (uint32_t)j & 1u;
+          const uint32_t acc = j > 0 ? 1u : 0u;
           const bool more = j + 1 < n_kv;
           if (!wait_phase(bar(kBarKVFull + slot_of(tv)), ph_of(tv), ctl)) break;
+          if (!wait_phase(bar(kBarPHalf + 0), par, ctl)) break;
+          tc_fence_after();
+          issue_pv_half<0>(tO[0], tS[0], vd, acc);
           if (!wait_phase(bar(kBarPFull + 0), par, ctl)) break;
           tc_fence_after();
-          issue_pv(tO[0], tS[0], vs, j > 0);
+          issue_pv_half<1>(tO[0], tS[0], vd, acc);
           if (more) {
             if (!wait_phase(bar(kBarKVFull + slot_of(tk)), ph_of(tk), ctl)) break;
             tc_fence_after();
-            issue_qk(tS[0], sQ, ks);
+            issue_qk(tS[0], dq0, kd);
             mma_commit(bar(kBarSFull + 0));
           } else {
             mma_commit(bar(kBarOFull + 0));
           }
+          if (!wait_phase(bar(kBarPHalf + 1), par, ctl)) break;
+          tc_fence_after();
+          issue_pv_half<0>(tO[1], tS[1], vd, acc);
           if (!wait_phase(bar(kBarPFull + 1), par, ctl)) break;
           tc_fence_after();
-          issue_pv(tO[1], tS[1], vs, j > 0);
+          issue_pv_half<1>(tO[1], tS[1], vd, acc);
           mma_commit(bar(kBarKVEmpty + slot_of(tv)));
           if (more) {
-            issue_qk(tS[1], sQ + kTileBytes, ks);
+            issue_qk(tS[1], dq1, kd);
             mma_commit(bar(kBarSFull + 1));
             mma_commit(bar(kBarKVEmpty + slot_of(tk)));
           } else {
@@ -402,32 +513,47 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           break;
         }
         tc_fence_after();
+        // S row in two halves: the max of the first half overlaps the load
+        // of the second.
         uint32_t sr[128];
         tmem::ld32(tS + 0, sr + 0);
         tmem::ld32(tS + 32, sr + 32);
+        tmem::wait_ld64(sr);
         tmem::ld32(tS + 64, sr + 64);
         tmem::ld32(tS + 96, sr + 96);
-        tmem::wait_ld128(sr);
         float *sv = reinterpret_cast<float *>(sr);
         const int64_t rem = len - (int64_t)kt * kBN;
-        if (rem < kBN) {
-          const int valid = (int)rem;
+        const int valid = rem < kBN ? (int)rem : kBN;
+        if (valid < kBN) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c >= valid) sv[c] = -INFINITY;
         }
-        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
+        float mA = -INFINITY, mB = -INFINITY, mC = -INFINITY, mD = -INFINITY;
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          m0 = fmaxf(m0, sv[c]);
-          m1 = fmaxf(m1, sv[c + 1]);
-          m2 = fmaxf(m2, sv[c + 2]);
-          m3 = fmaxf(m3, sv[c + 3]);
+        for (int c = 0; c < 64; c += 8) {
+          mA = fmax3(mA, sv[c], sv[c + 1]);
+          mB = fmax3(mB, sv[c + 2], sv[c + 3]);
+          mC = fmax3(mC, sv[c + 4], sv[c + 5]);
+          mD = fmax3(mD, sv[c + 6], sv[c + 7]);
         }
-        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+        tmem::wait_ld64(sr + 64);
+        if (valid < kBN) {
+#pragma unroll
+          for (int c = 64; c < 128; ++c)
+            if (c >= valid) sv[c] = -INFINITY;
+        }
+#pragma unroll
+        for (int c = 64; c < 128; c += 8) {
+          mA = fmax3(mA, sv[c], sv[c + 1]);
+          mB = fmax3(mB, sv[c + 2], sv[c + 3]);
+          mC = fmax3(mC, sv[c + 4], sv[c + 5]);
+          mD = fmax3(mD, sv[c + 6], sv[c + 7]);
+        }
+        const float mx = fmaxf(fmax3(mA, mB, mC), mD) * sl2;
         // Lazy max: raise it (and rescale O and l by alpha) only when some
-        // row of the warp grew by more than 2^8; the O update happens after
-        // P is stored, while the S values are no longer live.
+        // row of the warp grew by more than 2^8; the O update happens once
+        // the first half of P is stored, when its S values are no longer live.
         bool rescale = false;
         float alpha = 1.f;
         if (j == 0) {
@@ -439,20 +565,32 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           l *= alpha;
           rescale = true;
         }
-        const float neg_m = -m;
-        float l0 = 0.f, l1 = 0.f;
-        uint32_t pk[64];
+        // P = 2^(s * scale * log2 e - m) as bf16 pairs, published to the MMA
+        // lane in two halves of 64 keys so that O += P V on the first half
+        // overlaps the exponentials of the second.  The row sum accumulates
+        // the fp32 values.  A pending O rescale happens before the first
+        // half is published (the MMA lane may then start updating O).
+        const uint64_t sl2x2 = f2(sl2, sl2), negm2 = f2(-m, -m);
+        uint64_t lacc0 = f2(0.f, 0.f), lacc1 = f2(0.f, 0.f);
+        uint32_t pk0[32], pk1[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float e0 = ex2(fmaf(sv[2 * c], sl2, neg_m));
-          const float e1 = ex2(fmaf(sv[2 * c + 1], sl2, neg_m));
-          l0 += e0;
-          l1 += e1;
-          pk[c] = pack_bf16x2(e0, e1);
+        for (int c = 0; c < 32; ++c) {
+          const uint64_t x = fma2(f2(sv[2 * c], sv[2 * c + 1]), sl2x2, negm2);
+          uint64_t e;
+          if (pair_on_fma(c)) {
+            e = exp2_poly_x2(x);
+          } else {
+            const float2 xv = unf2(x);
+            e = f2(ex2(xv.x), ex2(xv.y));
+          }
+          if (c & 1)
+            lacc1 = add2(lacc1, e);
+          else
+            lacc0 = add2(lacc0, e);
+          const float2 ev = unf2(e);
+          pk0[c] = pack_bf16x2(ev.x, ev.y);
         }
-        l += l0 + l1;
-        tmem::st32(tS + 0, pk);
-        tmem::st32(tS + 32, pk + 32);
+        tmem::st32(tS + 0, pk0);
         if (rescale) {
 #pragma unroll
           for (int cc = 0; cc < 128; cc += 32) {
@@ -464,6 +602,31 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
               orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha);
             tmem::st32(tO + cc, orow);
           }
+        }
+        tmem::wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPHalf + tile));
+#pragma unroll
+        for (int c = 32; c < 64; ++c) {
+          const uint64_t x = fma2(f2(sv[2 * c], sv[2 * c + 1]), sl2x2, negm2);
+          uint64_t e;
+          if (pair_on_fma(c)) {
+            e = exp2_poly_x2(x);
+          } else {
+            const float2 xv = unf2(x);
+            e = f2(ex2(xv.x), ex2(xv.y));
+          }
+          if (c & 1)
+            lacc1 = add2(lacc1, e);
+          else
+            lacc0 = add2(lacc0, e);
+          const float2 ev = unf2(e);
+          pk1[c - 32] = pack_bf16x2(ev.x, ev.y);
+        }
+        tmem::st32(tS + 32, pk1);
+        {
+          const float2 a = unf2(lacc0), b = unf2(lacc1);
+          l += (a.x + a.y) + (b.x + b.y);
         }
         tmem::wait_st();
         tc_fence_before();

@@ -89,6 +89,10 @@ WORKLOADS = {
     # 720p-shaped: 30 frames of 23x40, 512 text tokens, 2 prior segments.
     "720p": Workload("720p", n_text=512, frames=30, grid_h=23, grid_w=40,
                      cache_frames=60, t0=60),
+    # Profiling-sized 720p grid: 8 frames over 15 cached frames (K/V 178 MB,
+    # above the 126 MB L2, so DRAM counters stay meaningful).
+    "short": Workload("short", n_text=512, frames=8, grid_h=23, grid_w=40,
+                      cache_frames=15, t0=15),
     # Bounded active history: 8 prior segments (240 frames) in the cache; a
     # 63-frame list is gathered into a window before the 720p attention.
     "bounded": Workload("bounded", n_text=512, frames=30, grid_h=23, grid_w=40,
