@@ -194,6 +194,46 @@ nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_
                                      int32_t heads, int32_t head_dim, int32_t *dev_err,
                                      void *stream);
 
+/*
+ * Power-spaced choice of the past latent frames to keep resident ("The 4090
+ * preset": N = min(budget, n_past), u_i = i/(N-1), d_i = i + rint((n_past -
+ * N) u_i^gamma), kept frames n_past - 1 - d_i; the page's preset uses budget
+ * 18 and gamma 2).  Host-only, no CUDA.
+ *   out     : host int32[out_capacity]; receives the N kept frames in
+ *             ascending order (frame 0, the oldest, is always kept when
+ *             n_past > 0).  *n_out = N.
+ * Errors: NOMAS_ERR_INVALID_ARG (negative counts, gamma < 0 or not finite,
+ * n_out NULL), NOMAS_ERR_CAPACITY (out_capacity < N).
+ */
+nomas_status nomas_temporal_context_frames(int32_t n_past, int32_t budget, float gamma,
+                                           int32_t *out, int32_t out_capacity, int32_t *n_out);
+
+/*
+ * Per-call options of nomas_segment_attention_ex.
+ *   wait_limit_ns: time limit of every pipeline wait inside the kernel
+ *                  (0 selects the default of 2 s).  A wait that runs out sets
+ *                  NOMAS_DEVERR_WAIT_TIMEOUT in *dev_err; the affected query
+ *                  block then writes no output, releases its resources and
+ *                  exits, and the CUDA context stays usable.
+ *   testing_skip_kv_load: -1 in normal use.  For tests of the timeout path
+ *                  only: a value k >= 0 makes every block leave out its k-th
+ *                  K/V tile load (loads alternate K, V, K, V ... over the key
+ *                  tiles), so a consumer wait cannot complete and must time out.
+ */
+typedef struct {
+  uint64_t wait_limit_ns;
+  int32_t testing_skip_kv_load;
+} nomas_attention_opts;
+
+/*
+ * nomas_segment_attention with per-call options (opts may be NULL for the
+ * defaults); identical otherwise.
+ */
+nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                        int32_t n_spans, void *o, float *lse, float softmax_scale,
+                                        int32_t heads, int32_t head_dim, int32_t *dev_err,
+                                        const nomas_attention_opts *opts, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

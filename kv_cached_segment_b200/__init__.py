@@ -39,6 +39,8 @@ EXPORTED_SYMBOLS = (
     "nomas_kvcache_append",
     "nomas_kvcache_select",
     "nomas_segment_attention",
+    "nomas_segment_attention_ex",
+    "nomas_temporal_context_frames",
 )
 
 
@@ -66,6 +68,10 @@ class _KVCache(ctypes.Structure):
 
 class _KVSpan(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64)]
+
+
+class _AttnOpts(ctypes.Structure):
+    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("testing_skip_kv_load", ctypes.c_int32)]
 
 
 _lib = None
@@ -102,6 +108,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_segment_attention.restype = ctypes.c_int
     lib.nomas_segment_attention.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, F32,
                                             I32, I32, P, P]
+    lib.nomas_segment_attention_ex.restype = ctypes.c_int
+    lib.nomas_segment_attention_ex.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, F32,
+                                               I32, I32, P, ctypes.POINTER(_AttnOpts), P]
+    lib.nomas_temporal_context_frames.restype = ctypes.c_int
+    lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
     return lib
 
@@ -233,6 +244,18 @@ def kvcache_append(cache: KVCache, k_seg, v_seg, q_in=None, q_out=None,
                                     _stream(stream)))
 
 
+def temporal_context_frames(n_past: int, budget: int = 18, gamma: float = 2.0) -> list:
+    """Past latent frames to keep resident (power-spaced back from the newest)."""
+    lib = load_library()
+    n = max(0, min(int(budget), int(n_past)))
+    out = (ctypes.c_int32 * max(1, n))()
+    n_out = ctypes.c_int32(0)
+    _check(lib.nomas_temporal_context_frames(int(n_past), int(budget), float(gamma),
+                                             ctypes.cast(out, ctypes.c_void_p), max(1, n),
+                                             ctypes.byref(n_out)))
+    return [int(out[i]) for i in range(n_out.value)]
+
+
 def kvcache_select(src: KVCache, frame_idx, window: KVCache, dev_err=None, stream=None) -> None:
     """Gathers the listed latent frames of ``src`` into ``window`` (bit-exact)."""
     lib = load_library()
@@ -253,8 +276,12 @@ def kvcache_select(src: KVCache, frame_idx, window: KVCache, dev_err=None, strea
 
 
 def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, dev_err=None,
-                      stream=None):
-    """Attention of every row of q over all keys of ``spans`` (list of (k, v)); returns o."""
+                      stream=None, wait_limit_ns: int = 0, testing_skip_kv_load: int = -1):
+    """Attention of every row of q over all keys of ``spans`` (list of (k, v)); returns o.
+
+    ``wait_limit_ns`` bounds every pipeline wait in the kernel (0: default);
+    ``testing_skip_kv_load`` is for tests of the timeout path only.
+    """
     lib = load_library()
     n_q = _rows(q, "q")
     if o is None:
@@ -273,7 +300,13 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
     if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
         raise TypeError("dev_err must be a CUDA int32 tensor")
-    _check(lib.nomas_segment_attention(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
-                                       float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
-                                       _stream(stream)))
+    if wait_limit_ns or testing_skip_kv_load != -1:
+        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load))
+        _check(lib.nomas_segment_attention_ex(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
+                                              float(softmax_scale), HEADS, HEAD_DIM,
+                                              _ptr(dev_err), ctypes.byref(opts), _stream(stream)))
+    else:
+        _check(lib.nomas_segment_attention(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
+                                           float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
+                                           _stream(stream)))
     return o

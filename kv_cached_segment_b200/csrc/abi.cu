@@ -322,6 +322,14 @@ nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_
                                      int32_t n_spans, void *o, float *lse, float softmax_scale,
                                      int32_t heads, int32_t head_dim, int32_t *dev_err,
                                      void *stream) {
+  return nomas_segment_attention_ex(q, n_q, spans, n_spans, o, lse, softmax_scale, heads, head_dim,
+                                    dev_err, nullptr, stream);
+}
+
+nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                        int32_t n_spans, void *o, float *lse, float softmax_scale,
+                                        int32_t heads, int32_t head_dim, int32_t *dev_err,
+                                        const nomas_attention_opts *opts, void *stream) {
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   if (n_spans < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_spans < 0");
@@ -373,6 +381,13 @@ nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_
   a.lse = lse;
   a.dev_err = dev_err;
   a.wait_limit_ns = g_wait_limit_ns;
+  a.testing_skip_load = -1;
+  if (opts != nullptr) {
+    if (opts->wait_limit_ns > 0) a.wait_limit_ns = opts->wait_limit_ns;
+    if (opts->testing_skip_kv_load < -1)
+      return fail(NOMAS_ERR_INVALID_ARG, "testing_skip_kv_load must be >= -1");
+    a.testing_skip_load = opts->testing_skip_kv_load;
+  }
   const cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();

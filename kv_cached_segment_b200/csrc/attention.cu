@@ -302,8 +302,12 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
 #ifndef NOMAS_EXP2_FMA_PAIRS
 #define NOMAS_EXP2_FMA_PAIRS 2
 #endif
+#ifndef NOMAS_EXP2_FMA_PAIRS_H1
+#define NOMAS_EXP2_FMA_PAIRS_H1 NOMAS_EXP2_FMA_PAIRS
+#endif
+// c < 32: first half of the tile (on the critical path to the MMA lane).
 __device__ __forceinline__ constexpr bool pair_on_fma(int c) {
-  return (c & 7) < NOMAS_EXP2_FMA_PAIRS;
+  return c < 32 ? (c & 7) < NOMAS_EXP2_FMA_PAIRS : (c & 7) < NOMAS_EXP2_FMA_PAIRS_H1;
 }
 
 // The MMA lane must issue an instruction every 64 cycles to keep the tensor
@@ -409,6 +413,9 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
         const int nt = num_tiles(p.span_len[s]);
         for (int kt = 0; kt < nt && ok; ++kt) {
           for (int which = 0; which < 2; ++which, ++t) {
+            // Testing hook: leave one load out so that a consumer wait runs
+            // out of time (exercises the bounded-wait abort path).
+            if (t == p.testing_skip_load) continue;
             const int slot = t % kStages;
             const uint32_t ph = (uint32_t)(t / kStages) & 1u;
             if (!wait_phase(bar(kBarKVEmpty + slot), ph ^ 1u, ctl)) {
@@ -426,7 +433,8 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       // Teardown: wait until every load this lane issued has landed.
       drain_phase(bar(kBarQFull), 0, p.wait_limit_ns);
       for (int u = (t > kStages ? t - kStages : 0); u < t; ++u)
-        drain_phase(bar(kBarKVFull + u % kStages), (uint32_t)(u / kStages) & 1u, p.wait_limit_ns);
+        if (u != p.testing_skip_load)
+          drain_phase(bar(kBarKVFull + u % kStages), (uint32_t)(u / kStages) & 1u, p.wait_limit_ns);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -508,7 +516,10 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       const int64_t len = p.span_len[s];
       const int nt = num_tiles(len);
       for (int kt = 0; kt < nt; ++kt, ++j) {
-        if (!wait_phase(bar(kBarSFull + tile), (uint32_t)j & 1u, ctl)) {
+        // Warp-uniform outcome: the tcgen05 loads and stores below are
+        // warp-collective, so a lane that saw the abort flag takes the whole
+        // warp with it.
+        if (!__all_sync(0xffffffffu, wait_phase(bar(kBarSFull + tile), (uint32_t)j & 1u, ctl))) {
           ok = false;
           break;
         }
@@ -634,7 +645,9 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       }
     }
     // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l).
-    if (ok && n_kv > 0 && wait_phase(bar(kBarOFull + tile), 0, ctl)) {
+    bool have_o = ok && n_kv > 0;
+    if (have_o) have_o = __all_sync(0xffffffffu, wait_phase(bar(kBarOFull + tile), 0, ctl));
+    if (have_o) {
       tc_fence_after();
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       const float inv_l = 1.0f / l;

@@ -66,6 +66,7 @@ struct AttnArgs {
   float scale_log2;            // softmax scale * log2(e)
   int32_t *dev_err;            // may be null
   unsigned long long wait_limit_ns;
+  int32_t testing_skip_load;   // -1, or the K/V load index the producer leaves out
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,

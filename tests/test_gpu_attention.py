@@ -188,3 +188,23 @@ def test_layer_step_bounded_sampled_rows():
     assert_close(f64(o[torch.as_tensor(rows)]), o_ref, what="bounded O")
     got_l = lse.view(16, -1)[:, torch.as_tensor(rows).cuda()].cpu().numpy().astype(np.float64)
     assert_close(got_l, l_ref, what="bounded LSE")
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    # The producer leaves out one K/V load, so a consumer wait can never
+    # complete: the kernel must give up after its (short) limit, report
+    # NOMAS_DEVERR_WAIT_TIMEOUT and leave the context usable.
+    q = randn_bf16((112, 16, 128), 1)
+    spans = [(randn_bf16((48, 16, 128), 2), randn_bf16((48, 16, 128), 3)),
+             (randn_bf16((64, 16, 128), 4), randn_bf16((64, 16, 128), 5)),
+             (randn_bf16((48, 16, 128), 6), randn_bf16((48, 16, 128), 7))]
+    sd = [(k.cuda(), v.cuda()) for k, v in spans]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = torch.full((112, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    nm.segment_attention(q.cuda(), sd, o=o, dev_err=err, wait_limit_ns=50_000_000,
+                         testing_skip_kv_load=3)
+    torch.cuda.synchronize()
+    assert int(err.item()) == nm.DEVERR_WAIT_TIMEOUT
+    assert torch.all(o == 7.0)  # aborted blocks write no output
+    # the same context still computes correct results
+    _check(q, spans, what="after timeout")
