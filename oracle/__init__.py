@@ -21,4 +21,7 @@ from .nomas_oracle import (  # noqa: F401
     attention,
     attention_rows,
     temporal_context_frame_indices,
+    f32_to_bf16_bits,
+    quantize_int8,
+    dequantize_int8,
 )

@@ -215,3 +215,47 @@ def temporal_context_frame_indices(n_past: int, budget: int = 18,
         d = i + int(np.rint((t - n) * u ** gamma))
         kept.append(t - 1 - d)
     return np.array(sorted(kept), dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
+# INT8 KV cache
+# ---------------------------------------------------------------------------
+def f32_to_bf16_bits(x) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even); bits.
+
+    bf16 keeps the upper 16 bits of a float32; rounding adds half of the
+    dropped part, plus one when the kept part is odd and the dropped part is
+    exactly half (ties to even).  Inputs are finite here.
+    """
+    b = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (b >> np.uint64(16)) & np.uint64(1)
+    rounded = (b + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
+    return rounded.astype(np.uint16)
+
+
+def quantize_int8(x_bits):
+    """Symmetric INT8 quantisation per (token, head) of a bf16 [N][H][D] tensor.
+
+    [KV] "The 4090 preset": the cache is quantised once per segment to one
+    byte per value plus an FP32 scale per token and head (4,224 B per token
+    per layer for K and V together).  Reading (the page gives no formula):
+    absmax scaling in float32, scale = max_d |x_d| / 127 and code =
+    rint(x_d / scale), both divisions rounded to nearest in float32 and rint
+    rounding half to even; an all-zero (token, head) gets scale 0 and codes 0.
+    Returns int8 codes [N][H][D] and float32 scales [N][H].
+    """
+    x = bf16_bits_to_f64(x_bits).astype(np.float32)          # exact
+    amax = np.max(np.abs(x), axis=2)                           # exact
+    scale = (amax / np.float32(127.0)).astype(np.float32)      # fp32 RN
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (x / safe[:, :, None]).astype(np.float32)              # fp32 RN
+    codes = np.clip(np.rint(q), -127, 127).astype(np.int8)
+    codes[scale == 0] = 0
+    return codes, scale
+
+
+def dequantize_int8(codes, scales) -> np.ndarray:
+    """bf16 bits of code * scale (product in float32, then rounded to bf16)."""
+    prod = (np.asarray(codes, dtype=np.float32) *
+            np.asarray(scales, dtype=np.float32)[:, :, None]).astype(np.float32)
+    return f32_to_bf16_bits(prod)

@@ -351,3 +351,58 @@ def test_picker_keeps_first_and_newest_frames(t):
 
 def test_picker_empty_history():
     assert O.temporal_context_frame_indices(0).size == 0
+
+
+# ------------------------------------------------------------- INT8 cache --
+def _bits_of(x):
+    return O.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def test_bf16_rounding_known_patterns():
+    # 1 + 2^-8 is a tie between 0x3F80 and 0x3F81: ties go to the even 0x3F80;
+    # 1 + 3*2^-8 ties between 0x3F81 and 0x3F82: to even 0x3F82; 1 + 2^-7 is
+    # exact (0x3F81); just above a tie rounds up.
+    vals = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -7, 1.0 + 2 ** -8 + 2 ** -20, -2.5, 0.0]
+    assert _bits_of(vals).tolist() == [0x3F80, 0x3F82, 0x3F81, 0x3F81, 0xC020, 0x0000]
+
+
+def test_int8_layout_bytes_match_page(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "cache_sizes.json")))
+    x = _bits_of(np.ones((3, g["heads"], g["head_dim"])))
+    codes, scales = O.quantize_int8(x)
+    per_token = 2 * (codes[0].nbytes + scales[0].nbytes)  # K and V
+    assert per_token == g["int8_bytes_per_token_layer"]
+
+
+def test_int8_absmax_maps_to_127_and_sign_symmetry():
+    r = rng(20)
+    x = _bits_of(r.standard_normal((50, 4, 128)) * 3)
+    codes, scales = O.quantize_int8(x)
+    xf = O.bf16_bits_to_f64(x)
+    am = np.argmax(np.abs(xf), axis=2)
+    top = np.take_along_axis(codes, am[:, :, None], axis=2)[:, :, 0].astype(int)
+    assert np.all(np.abs(top) == 127)
+    neg = O.quantize_int8(x ^ np.uint16(0x8000))  # flip every sign bit
+    assert np.array_equal(neg[0], -codes) and np.array_equal(neg[1], scales)
+
+
+def test_int8_error_bound_and_exact_grid():
+    r = rng(21)
+    x = _bits_of(r.standard_normal((40, 2, 128)))
+    codes, scales = O.quantize_int8(x)
+    xf = O.bf16_bits_to_f64(x)
+    deq = O.bf16_bits_to_f64(O.dequantize_int8(codes, scales))
+    bound = 0.5 * scales[:, :, None] * (1 + 1e-6) + np.abs(xf) * 2.0 ** -8 + 1e-30
+    assert np.all(np.abs(deq - xf) <= bound)
+    # values that are exact multiples of a power-of-two step come back exactly
+    grid = np.arange(-127, 129)[:128].reshape(1, 1, 128) * 2.0 ** -4
+    g = _bits_of(grid)
+    c2, s2 = O.quantize_int8(g)
+    assert np.array_equal(O.dequantize_int8(c2, s2), g)
+
+
+def test_int8_zero_rows():
+    z = np.zeros((2, 3, 128), dtype=np.uint16)
+    codes, scales = O.quantize_int8(z)
+    assert np.all(codes == 0) and np.all(scales == 0)
+    assert np.all(O.dequantize_int8(codes, scales) == 0)
