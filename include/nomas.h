@@ -195,6 +195,43 @@ nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_
                                      void *stream);
 
 /*
+ * INT8 layer cache ("The 4090 preset": the cache is quantised once per
+ * segment to one byte per value plus an FP32 scale per token and head, 4,224
+ * B per token per layer for K and V together).  k and v hold int8 codes
+ * [capacity][heads][head_dim]; k_scale and v_scale hold fp32 [capacity][heads].
+ * Value = code * scale.  Caller-owned device memory, 16-byte aligned.
+ */
+typedef struct {
+  void *k, *v;
+  float *k_scale, *v_scale;
+  int64_t capacity, len;
+  int32_t tokens_per_frame, heads, head_dim;
+} nomas_kvcache_i8;
+
+/*
+ * nomas_kvcache_append into an INT8 cache: the rotated segment keys (rounded
+ * to bf16, as the bf16 path would store them) and the values are quantised
+ * per (token, head) with scale = absmax / 127 and code = rint(x / scale),
+ * both divisions rounded to nearest in fp32 and rint rounding half to even;
+ * an all-zero (token, head) gets scale 0 and codes 0.  Q is handled exactly as
+ * in nomas_kvcache_append.  Same errors as nomas_kvcache_append.
+ */
+nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
+                                     const void *v_seg, int64_t n_tokens, const void *q_in,
+                                     void *q_out, const nomas_seg_layout *layout,
+                                     const nomas_rope3d_cfg *cfg, void *stream);
+
+/*
+ * nomas_kvcache_select from an INT8 cache into a bf16 window: the listed
+ * frames are restored to the GPU-side window as bf16(fp32(code * scale))
+ * (product rounded to nearest in fp32, then to bf16 nearest-even).  Same
+ * arguments, index checks and errors as nomas_kvcache_select.
+ */
+nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
+                                     int32_t n_frames, int32_t idx_on_device,
+                                     nomas_kvcache *window, int32_t *dev_err, void *stream);
+
+/*
  * Power-spaced choice of the past latent frames to keep resident ("The 4090
  * preset": N = min(budget, n_past), u_i = i/(N-1), d_i = i + rint((n_past -
  * N) u_i^gamma), kept frames n_past - 1 - d_i; the page's preset uses budget

@@ -41,6 +41,8 @@ EXPORTED_SYMBOLS = (
     "nomas_segment_attention",
     "nomas_segment_attention_ex",
     "nomas_temporal_context_frames",
+    "nomas_kvcache_append_i8",
+    "nomas_kvcache_select_i8",
 )
 
 
@@ -62,6 +64,13 @@ class _SegLayout(ctypes.Structure):
 
 class _KVCache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("capacity", ctypes.c_int64),
+                ("len", ctypes.c_int64), ("tokens_per_frame", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class _KVCacheI8(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("capacity", ctypes.c_int64),
                 ("len", ctypes.c_int64), ("tokens_per_frame", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
@@ -111,6 +120,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_segment_attention_ex.restype = ctypes.c_int
     lib.nomas_segment_attention_ex.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, F32,
                                                I32, I32, P, ctypes.POINTER(_AttnOpts), P]
+    lib.nomas_kvcache_append_i8.restype = ctypes.c_int
+    lib.nomas_kvcache_append_i8.argtypes = [ctypes.POINTER(_KVCacheI8), P, P, I64, P, P,
+                                            ctypes.POINTER(_SegLayout), ctypes.POINTER(_RopeCfg),
+                                            P]
+    lib.nomas_kvcache_select_i8.restype = ctypes.c_int
+    lib.nomas_kvcache_select_i8.argtypes = [ctypes.POINTER(_KVCacheI8), P, I32, I32,
+                                            ctypes.POINTER(_KVCache), P, P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -209,6 +225,61 @@ class KVCache:
         return self.k[start:stop], self.v[start:stop]
 
 
+class KVCacheI8:
+    """INT8 layer cache: int8 codes [capacity][16][128] and fp32 scales [capacity][16] for K and V."""
+
+    def __init__(self, k, v, k_scale, v_scale, length: int, tokens_per_frame: int):
+        for t, name in ((k, "k"), (v, "v")):
+            if t.dtype != torch.int8 or not t.is_cuda or not t.is_contiguous() or \
+                    t.dim() != 3 or t.shape[1:] != (HEADS, HEAD_DIM):
+                raise TypeError(f"INT8 cache {name} must be contiguous CUDA int8 [N][16][128]")
+        for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or \
+                    t.shape != (k.shape[0], HEADS):
+                raise TypeError(f"INT8 cache {name} must be contiguous CUDA fp32 [N][16]")
+        self.k, self.v, self.k_scale, self.v_scale = k, v, k_scale, v_scale
+        self._c = _KVCacheI8(k.data_ptr(), v.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(),
+                             k.shape[0], int(length), int(tokens_per_frame), HEADS, HEAD_DIM)
+
+    @classmethod
+    def empty(cls, capacity: int, tokens_per_frame: int, device="cuda"):
+        k = torch.empty((capacity, HEADS, HEAD_DIM), dtype=torch.int8, device=device)
+        s = torch.empty((capacity, HEADS), dtype=torch.float32, device=device)
+        return cls(k, torch.empty_like(k), s, torch.empty_like(s), 0, tokens_per_frame)
+
+    @property
+    def len(self) -> int:
+        return self._c.len
+
+    @len.setter
+    def len(self, n: int) -> None:
+        self._c.len = int(n)
+
+    @property
+    def capacity(self) -> int:
+        return self._c.capacity
+
+
+def kvcache_append_i8(cache: KVCacheI8, k_seg, v_seg, q_in=None, q_out=None,
+                      layout: SegLayout | None = None, cfg: RopeConfig | None = None,
+                      stream=None) -> None:
+    """kvcache_append into an INT8 cache (keys rotated, then K and V quantised)."""
+    lib = load_library()
+    n = _rows(k_seg, "k_seg")
+    if _rows(v_seg, "v_seg") != n:
+        raise ValueError("k_seg and v_seg differ in rows")
+    if q_in is not None:
+        _rows(q_in, "q_in")
+        _rows(q_out, "q_out")
+    lay = layout._c() if layout is not None else None
+    c = cfg._c() if cfg is not None else None
+    _check(lib.nomas_kvcache_append_i8(ctypes.byref(cache._c), _ptr(k_seg), _ptr(v_seg), n,
+                                       _ptr(q_in), _ptr(q_out),
+                                       ctypes.byref(lay) if lay is not None else None,
+                                       ctypes.byref(c) if c is not None else None,
+                                       _stream(stream)))
+
+
 def rope3d_qk(q, k, q_out, k_out, layout: SegLayout, cfg: RopeConfig, stream=None) -> None:
     """3D RoPE on Q (and K): video rows rotated, text rows copied."""
     lib = load_library()
@@ -256,8 +327,12 @@ def temporal_context_frames(n_past: int, budget: int = 18, gamma: float = 2.0) -
     return [int(out[i]) for i in range(n_out.value)]
 
 
-def kvcache_select(src: KVCache, frame_idx, window: KVCache, dev_err=None, stream=None) -> None:
-    """Gathers the listed latent frames of ``src`` into ``window`` (bit-exact)."""
+def kvcache_select(src, frame_idx, window: KVCache, dev_err=None, stream=None) -> None:
+    """Gathers the listed latent frames of ``src`` into the bf16 ``window``.
+
+    A bf16 ``src`` is copied bit for bit; an INT8 ``src`` (KVCacheI8) is
+    dequantised (code * scale, rounded to bf16).
+    """
     lib = load_library()
     if isinstance(frame_idx, torch.Tensor) and frame_idx.is_cuda:
         if frame_idx.dtype != torch.int32 or not frame_idx.is_contiguous():
@@ -270,8 +345,9 @@ def kvcache_select(src: KVCache, frame_idx, window: KVCache, dev_err=None, strea
         ptr = ctypes.cast(arr, ctypes.c_void_p).value
     if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
         raise TypeError("dev_err must be a CUDA int32 tensor")
-    _check(lib.nomas_kvcache_select(ctypes.byref(src._c), ptr, n, on_dev, ctypes.byref(window._c),
-                                    _ptr(dev_err), _stream(stream)))
+    fn = lib.nomas_kvcache_select_i8 if isinstance(src, KVCacheI8) else lib.nomas_kvcache_select
+    _check(fn(ctypes.byref(src._c), ptr, n, on_dev, ctypes.byref(window._c), _ptr(dev_err),
+              _stream(stream)))
     del keep
 
 

@@ -135,6 +135,181 @@ nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows) {
   return NOMAS_OK;
 }
 
+// A bf16 or INT8 layer cache seen by the append path.
+struct CacheView {
+  void *k, *v;
+  float *k_scale, *v_scale;  // INT8 only
+  int64_t capacity, len;
+  int32_t heads, head_dim;
+  bool int8;
+};
+
+nomas_status append_common(const CacheView &c, const void *k_seg, const void *v_seg,
+                           int64_t n_tokens, const void *q_in, void *q_out,
+                           const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
+                           void *stream) {
+  nomas_status st = check_shape(c.heads, c.head_dim);
+  if (st != NOMAS_OK) return st;
+  if (c.k == nullptr || c.v == nullptr || !aligned16(c.k) || !aligned16(c.v))
+    return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
+  if (c.int8 && (c.k_scale == nullptr || c.v_scale == nullptr || !aligned16(c.k_scale) ||
+                 !aligned16(c.v_scale)))
+    return fail(NOMAS_ERR_INVALID_ARG, "cache scales must be non-NULL and 16-byte aligned");
+  if (c.capacity < 0 || c.len < 0 || c.len > c.capacity)
+    return fail(NOMAS_ERR_INVALID_ARG, "cache len/capacity inconsistent (%lld/%lld)",
+                (long long)c.len, (long long)c.capacity);
+  if (n_tokens < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_tokens < 0");
+  if (n_tokens > 0 && (k_seg == nullptr || v_seg == nullptr))
+    return fail(NOMAS_ERR_INVALID_ARG, "k_seg and v_seg are required");
+  if ((q_in == nullptr) != (q_out == nullptr))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_in and q_out must both be set or both be NULL");
+  if (!aligned16(k_seg) || !aligned16(v_seg) || !aligned16(q_in) || !aligned16(q_out))
+    return fail(NOMAS_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  RopeArgs a{};
+  int64_t n_video = 0, n_text = 0;
+  if (layout != nullptr) {
+    if ((st = check_layout(layout, &n_video)) != NOMAS_OK) return st;
+    n_text = layout->n_text;
+  }
+  if (cfg != nullptr) {
+    if (layout == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "rope cfg given without a layout");
+    if ((st = fill_rope(cfg, &a)) != NOMAS_OK) return st;
+    if (n_video != n_tokens)
+      return fail(NOMAS_ERR_INVALID_ARG, "n_tokens (%lld) != frames*grid_h*grid_w (%lld)",
+                  (long long)n_tokens, (long long)n_video);
+  }
+  if (c.len + n_tokens > c.capacity)
+    return fail(NOMAS_ERR_CAPACITY, "append of %lld rows at len %lld exceeds capacity %lld",
+                (long long)n_tokens, (long long)c.len, (long long)c.capacity);
+  const int64_t q_rows = q_in != nullptr ? n_tokens + n_text : 0;
+  const int64_t elem = c.int8 ? 1 : 2;  // bytes per cached value
+  uint8_t *k_dst = static_cast<uint8_t *>(c.k) + c.len * kRowElems * elem;
+  uint8_t *v_dst = static_cast<uint8_t *>(c.v) + c.len * kRowElems * elem;
+  const int64_t seg_bytes = n_tokens * kRowBytes, q_bytes = q_rows * kRowBytes;
+  const int64_t dst_bytes = n_tokens * kRowElems * elem;
+  if (overlap(k_seg, seg_bytes, k_dst, dst_bytes) || overlap(v_seg, seg_bytes, v_dst, dst_bytes) ||
+      overlap(k_seg, seg_bytes, v_dst, dst_bytes) || overlap(v_seg, seg_bytes, k_dst, dst_bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "segment K/V overlap the cache rows being written");
+  if (q_in != nullptr && q_out != q_in && overlap(q_in, q_bytes, q_out, q_bytes))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_out partially overlaps q_in");
+  if (q_out != nullptr && (overlap(q_out, q_bytes, k_dst, dst_bytes) ||
+                           overlap(q_out, q_bytes, v_dst, dst_bytes)))
+    return fail(NOMAS_ERR_INVALID_ARG, "q_out overlaps the cache rows being written");
+  a.q_in = static_cast<const uint16_t *>(q_in);
+  a.q_out = static_cast<uint16_t *>(q_out);
+  a.k_in = static_cast<const uint16_t *>(k_seg);
+  a.v_in = static_cast<const uint16_t *>(v_seg);
+  if (c.int8) {
+    a.k_codes = reinterpret_cast<int8_t *>(k_dst);
+    a.v_codes = reinterpret_cast<int8_t *>(v_dst);
+    a.k_scales = c.k_scale + c.len * kHeads;
+    a.v_scales = c.v_scale + c.len * kHeads;
+  } else {
+    a.k_out = reinterpret_cast<uint16_t *>(k_dst);
+    a.v_out = reinterpret_cast<uint16_t *>(v_dst);
+  }
+  a.n_q_rows = q_rows;
+  a.n_kv_rows = n_tokens;
+  a.n_video = cfg != nullptr ? n_tokens : 0;
+  if (layout != nullptr) {
+    a.grid_h = layout->grid_h;
+    a.grid_w = layout->grid_w;
+    a.t0 = layout->t0;
+  }
+  if (q_rows > 0 || n_tokens > 0) {
+    const cudaError_t e = c.int8 ? launch_rope_append_i8(a, static_cast<cudaStream_t>(stream))
+                                 : launch_rope_append(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  return NOMAS_OK;
+}
+
+nomas_status select_common(const CacheView &src, int32_t tokens_per_frame,
+                           const int32_t *frame_idx, int32_t n_frames, int32_t idx_on_device,
+                           nomas_kvcache *window, int32_t *dev_err, void *stream) {
+  nomas_status st = check_shape(src.heads, src.head_dim);
+  if (st != NOMAS_OK) return st;
+  if ((st = check_shape(window->heads, window->head_dim)) != NOMAS_OK) return st;
+  if (tokens_per_frame <= 0) return fail(NOMAS_ERR_INVALID_ARG, "src tokens_per_frame <= 0");
+  if (n_frames < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_frames < 0");
+  if (src.len < 0 || src.len > src.capacity || window->capacity < 0)
+    return fail(NOMAS_ERR_INVALID_ARG, "src len/capacity inconsistent");
+  const int64_t P = tokens_per_frame;
+  const int64_t rows = (int64_t)n_frames * P;
+  if (rows > window->capacity)
+    return fail(NOMAS_ERR_CAPACITY, "window capacity %lld < %d frames x %lld rows",
+                (long long)window->capacity, n_frames, (long long)P);
+  if (n_frames > 0) {
+    if (frame_idx == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "frame_idx is NULL");
+    if (src.k == nullptr || src.v == nullptr || window->k == nullptr || window->v == nullptr ||
+        !aligned16(src.k) || !aligned16(src.v) || !aligned16(window->k) || !aligned16(window->v))
+      return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
+    if (src.int8 && (src.k_scale == nullptr || src.v_scale == nullptr ||
+                     !aligned16(src.k_scale) || !aligned16(src.v_scale)))
+      return fail(NOMAS_ERR_INVALID_ARG, "cache scales must be non-NULL and 16-byte aligned");
+    const int64_t sb = src.len * kRowElems * (src.int8 ? 1 : 2), wb = rows * kRowBytes;
+    if (overlap(src.k, sb, window->k, wb) || overlap(src.v, sb, window->v, wb) ||
+        overlap(src.k, sb, window->v, wb) || overlap(src.v, sb, window->k, wb) ||
+        overlap(window->k, wb, window->v, wb))
+      return fail(NOMAS_ERR_INVALID_ARG, "window overlaps the source cache");
+    if (src.int8) {
+      const int64_t scb = src.len * kHeads * 4;
+      if (overlap(src.k_scale, scb, window->k, wb) || overlap(src.k_scale, scb, window->v, wb) ||
+          overlap(src.v_scale, scb, window->k, wb) || overlap(src.v_scale, scb, window->v, wb))
+        return fail(NOMAS_ERR_INVALID_ARG, "window overlaps the source scales");
+    }
+  }
+  const int64_t n_src_frames = src.len / P;
+  if (idx_on_device && n_frames > 0 && dev_err == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "dev_err is required for a device-resident frame list");
+  if (!idx_on_device) {
+    for (int32_t j = 0; j < n_frames; ++j)
+      if (frame_idx[j] < 0 || frame_idx[j] >= n_src_frames)
+        return fail(NOMAS_ERR_INDEX, "frame_idx[%d] = %d outside [0, %lld)", j, frame_idx[j],
+                    (long long)n_src_frames);
+  }
+  const int chunk = idx_on_device ? 65535 : kSelectHostFramesPerLaunch;
+  SelectHostList hl;
+  for (int32_t f0 = 0; f0 < n_frames; f0 += chunk) {
+    const int32_t nf = (n_frames - f0) < chunk ? (n_frames - f0) : chunk;
+    if (!idx_on_device) std::memcpy(hl.idx, frame_idx + f0, sizeof(int32_t) * nf);
+    cudaError_t e;
+    if (src.int8) {
+      SelectI8Args a{};
+      a.src_k = static_cast<const int8_t *>(src.k);
+      a.src_v = static_cast<const int8_t *>(src.v);
+      a.src_ks = src.k_scale;
+      a.src_vs = src.v_scale;
+      a.dst_k = static_cast<uint16_t *>(window->k);
+      a.dst_v = static_cast<uint16_t *>(window->v);
+      a.idx_dev = idx_on_device ? frame_idx : nullptr;
+      a.dev_err = dev_err;
+      a.tokens_per_frame = P;
+      a.n_src_frames = n_src_frames;
+      a.first_frame = f0;
+      a.n_frames = nf;
+      e = launch_select_i8(a, idx_on_device ? nullptr : &hl, static_cast<cudaStream_t>(stream));
+    } else {
+      SelectArgs a{};
+      a.src_k = static_cast<const uint16_t *>(src.k);
+      a.src_v = static_cast<const uint16_t *>(src.v);
+      a.dst_k = static_cast<uint16_t *>(window->k);
+      a.dst_v = static_cast<uint16_t *>(window->v);
+      a.idx_dev = idx_on_device ? frame_idx : nullptr;
+      a.dev_err = dev_err;
+      a.frame_vecs = P * kRowVecs;
+      a.n_src_frames = n_src_frames;
+      a.first_frame = f0;
+      a.n_frames = nf;
+      e = launch_select(a, idx_on_device ? nullptr : &hl, static_cast<cudaStream_t>(stream));
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  }
+  window->tokens_per_frame = tokens_per_frame;
+  window->len = rows;
+  return ok();
+}
+
 unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s per pipeline wait
 
 }  // namespace
@@ -189,66 +364,25 @@ nomas_status nomas_kvcache_append(nomas_kvcache *cache, const void *k_seg, const
                                   const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
                                   void *stream) {
   if (cache == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "cache is NULL");
-  nomas_status st = check_shape(cache->heads, cache->head_dim);
+  CacheView view{cache->k, cache->v, nullptr, nullptr, cache->capacity, cache->len,
+                 cache->heads, cache->head_dim, false};
+  const nomas_status st =
+      append_common(view, k_seg, v_seg, n_tokens, q_in, q_out, layout, cfg, stream);
   if (st != NOMAS_OK) return st;
-  if (cache->k == nullptr || cache->v == nullptr || !aligned16(cache->k) || !aligned16(cache->v))
-    return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
-  if (cache->capacity < 0 || cache->len < 0 || cache->len > cache->capacity)
-    return fail(NOMAS_ERR_INVALID_ARG, "cache len/capacity inconsistent (%lld/%lld)",
-                (long long)cache->len, (long long)cache->capacity);
-  if (n_tokens < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_tokens < 0");
-  if (n_tokens > 0 && (k_seg == nullptr || v_seg == nullptr))
-    return fail(NOMAS_ERR_INVALID_ARG, "k_seg and v_seg are required");
-  if ((q_in == nullptr) != (q_out == nullptr))
-    return fail(NOMAS_ERR_INVALID_ARG, "q_in and q_out must both be set or both be NULL");
-  if (!aligned16(k_seg) || !aligned16(v_seg) || !aligned16(q_in) || !aligned16(q_out))
-    return fail(NOMAS_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  RopeArgs a{};
-  int64_t n_video = 0, n_text = 0;
-  if (layout != nullptr) {
-    if ((st = check_layout(layout, &n_video)) != NOMAS_OK) return st;
-    n_text = layout->n_text;
-  }
-  if (cfg != nullptr) {
-    if (layout == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "rope cfg given without a layout");
-    if ((st = fill_rope(cfg, &a)) != NOMAS_OK) return st;
-    if (n_video != n_tokens)
-      return fail(NOMAS_ERR_INVALID_ARG, "n_tokens (%lld) != frames*grid_h*grid_w (%lld)",
-                  (long long)n_tokens, (long long)n_video);
-  }
-  if (cache->len + n_tokens > cache->capacity)
-    return fail(NOMAS_ERR_CAPACITY, "append of %lld rows at len %lld exceeds capacity %lld",
-                (long long)n_tokens, (long long)cache->len, (long long)cache->capacity);
-  const int64_t q_rows = q_in != nullptr ? n_tokens + n_text : 0;
-  uint16_t *k_dst = static_cast<uint16_t *>(cache->k) + cache->len * kRowElems;
-  uint16_t *v_dst = static_cast<uint16_t *>(cache->v) + cache->len * kRowElems;
-  const int64_t seg_bytes = n_tokens * kRowBytes, q_bytes = q_rows * kRowBytes;
-  if (overlap(k_seg, seg_bytes, k_dst, seg_bytes) || overlap(v_seg, seg_bytes, v_dst, seg_bytes) ||
-      overlap(k_seg, seg_bytes, v_dst, seg_bytes) || overlap(v_seg, seg_bytes, k_dst, seg_bytes))
-    return fail(NOMAS_ERR_INVALID_ARG, "segment K/V overlap the cache rows being written");
-  if (q_in != nullptr && q_out != q_in && overlap(q_in, q_bytes, q_out, q_bytes))
-    return fail(NOMAS_ERR_INVALID_ARG, "q_out partially overlaps q_in");
-  if (q_out != nullptr && (overlap(q_out, q_bytes, k_dst, seg_bytes) ||
-                           overlap(q_out, q_bytes, v_dst, seg_bytes)))
-    return fail(NOMAS_ERR_INVALID_ARG, "q_out overlaps the cache rows being written");
-  a.q_in = static_cast<const uint16_t *>(q_in);
-  a.q_out = static_cast<uint16_t *>(q_out);
-  a.k_in = static_cast<const uint16_t *>(k_seg);
-  a.k_out = k_dst;
-  a.v_in = static_cast<const uint16_t *>(v_seg);
-  a.v_out = v_dst;
-  a.n_q_rows = q_rows;
-  a.n_kv_rows = n_tokens;
-  a.n_video = cfg != nullptr ? n_tokens : 0;
-  if (layout != nullptr) {
-    a.grid_h = layout->grid_h;
-    a.grid_w = layout->grid_w;
-    a.t0 = layout->t0;
-  }
-  if (q_rows > 0 || n_tokens > 0) {
-    const cudaError_t e = launch_rope_append(a, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "append launch");
-  }
+  cache->len += n_tokens;
+  return ok();
+}
+
+nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
+                                     const void *v_seg, int64_t n_tokens, const void *q_in,
+                                     void *q_out, const nomas_seg_layout *layout,
+                                     const nomas_rope3d_cfg *cfg, void *stream) {
+  if (cache == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "cache is NULL");
+  CacheView view{cache->k, cache->v, cache->k_scale, cache->v_scale, cache->capacity,
+                 cache->len, cache->heads, cache->head_dim, true};
+  const nomas_status st =
+      append_common(view, k_seg, v_seg, n_tokens, q_in, q_out, layout, cfg, stream);
+  if (st != NOMAS_OK) return st;
   cache->len += n_tokens;
   return ok();
 }
@@ -257,65 +391,20 @@ nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame
                                   int32_t n_frames, int32_t idx_on_device, nomas_kvcache *window,
                                   int32_t *dev_err, void *stream) {
   if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
-  nomas_status st = check_shape(src->heads, src->head_dim);
-  if (st != NOMAS_OK) return st;
-  if ((st = check_shape(window->heads, window->head_dim)) != NOMAS_OK) return st;
-  if (src->tokens_per_frame <= 0) return fail(NOMAS_ERR_INVALID_ARG, "src tokens_per_frame <= 0");
-  if (n_frames < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_frames < 0");
-  if (src->len < 0 || src->len > src->capacity || window->capacity < 0)
-    return fail(NOMAS_ERR_INVALID_ARG, "src len/capacity inconsistent");
-  const int64_t P = src->tokens_per_frame;
-  const int64_t rows = (int64_t)n_frames * P;
-  if (rows > window->capacity)
-    return fail(NOMAS_ERR_CAPACITY, "window capacity %lld < %d frames x %lld rows",
-                (long long)window->capacity, n_frames, (long long)P);
-  if (n_frames > 0) {
-    if (frame_idx == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "frame_idx is NULL");
-    if (src->k == nullptr || src->v == nullptr || window->k == nullptr || window->v == nullptr ||
-        !aligned16(src->k) || !aligned16(src->v) || !aligned16(window->k) || !aligned16(window->v))
-      return fail(NOMAS_ERR_INVALID_ARG, "cache k/v must be non-NULL and 16-byte aligned");
-    const int64_t sb = src->len * kRowBytes, wb = rows * kRowBytes;
-    if (overlap(src->k, sb, window->k, wb) || overlap(src->v, sb, window->v, wb) ||
-        overlap(src->k, sb, window->v, wb) || overlap(src->v, sb, window->k, wb) ||
-        overlap(window->k, wb, window->v, wb))
-      return fail(NOMAS_ERR_INVALID_ARG, "window overlaps the source cache");
-  }
-  const int64_t n_src_frames = src->len / P;
-  if (idx_on_device && n_frames > 0 && dev_err == nullptr)
-    return fail(NOMAS_ERR_INVALID_ARG, "dev_err is required for a device-resident frame list");
-  if (!idx_on_device) {
-    for (int32_t j = 0; j < n_frames; ++j)
-      if (frame_idx[j] < 0 || frame_idx[j] >= n_src_frames)
-        return fail(NOMAS_ERR_INDEX, "frame_idx[%d] = %d outside [0, %lld)", j, frame_idx[j],
-                    (long long)n_src_frames);
-  }
-  SelectArgs a{};
-  a.src_k = static_cast<const uint16_t *>(src->k);
-  a.src_v = static_cast<const uint16_t *>(src->v);
-  a.dst_k = static_cast<uint16_t *>(window->k);
-  a.dst_v = static_cast<uint16_t *>(window->v);
-  a.dev_err = dev_err;
-  a.frame_vecs = P * kRowVecs;
-  a.n_src_frames = n_src_frames;
-  const int chunk = idx_on_device ? 65535 : kSelectHostFramesPerLaunch;
-  SelectHostList hl;
-  for (int32_t f0 = 0; f0 < n_frames; f0 += chunk) {
-    const int32_t nf = (n_frames - f0) < chunk ? (n_frames - f0) : chunk;
-    a.first_frame = f0;
-    a.n_frames = nf;
-    if (idx_on_device) {
-      a.idx_dev = frame_idx;
-    } else {
-      a.idx_dev = nullptr;
-      std::memcpy(hl.idx, frame_idx + f0, sizeof(int32_t) * nf);
-    }
-    const cudaError_t e =
-        launch_select(a, idx_on_device ? nullptr : &hl, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "select launch");
-  }
-  window->tokens_per_frame = src->tokens_per_frame;
-  window->len = rows;
-  return ok();
+  CacheView view{src->k, src->v, nullptr, nullptr, src->capacity, src->len,
+                 src->heads, src->head_dim, false};
+  return select_common(view, src->tokens_per_frame, frame_idx, n_frames, idx_on_device, window,
+                       dev_err, stream);
+}
+
+nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
+                                     int32_t n_frames, int32_t idx_on_device,
+                                     nomas_kvcache *window, int32_t *dev_err, void *stream) {
+  if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
+  CacheView view{src->k, src->v, src->k_scale, src->v_scale, src->capacity, src->len,
+                 src->heads, src->head_dim, true};
+  return select_common(view, src->tokens_per_frame, frame_idx, n_frames, idx_on_device, window,
+                       dev_err, stream);
 }
 
 nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_span *spans,

@@ -31,8 +31,13 @@ struct RopeArgs {
   // (0 = t, 1 = h, 2 = w) of the 64 rotation pairs of a head.
   double omega[kHeadDim / 2];
   int8_t axis[kHeadDim / 2];
+  // INT8 cache output (used by launch_rope_append_i8 instead of k_out/v_out):
+  // codes [rows][16][128] int8 and scales [rows][16] fp32, per token and head.
+  int8_t *k_codes, *v_codes;
+  float *k_scales, *v_scales;
 };
 cudaError_t launch_rope_append(const RopeArgs &a, cudaStream_t stream);
+cudaError_t launch_rope_append_i8(const RopeArgs &a, cudaStream_t stream);
 
 // -------------------------------------------------------------- select ----
 constexpr int kSelectHostFramesPerLaunch = 2048;
@@ -51,6 +56,20 @@ struct SelectHostList {
 };
 cudaError_t launch_select(const SelectArgs &a, const SelectHostList *host_list,
                           cudaStream_t stream);
+// Gather + dequantize from an INT8 cache into a bf16 window.
+struct SelectI8Args {
+  const int8_t *src_k, *src_v;        // codes [rows][16][128]
+  const float *src_ks, *src_vs;       // scales [rows][16]
+  uint16_t *dst_k, *dst_v;            // bf16 [rows][16][128]
+  const int32_t *idx_dev;
+  int32_t *dev_err;
+  int64_t tokens_per_frame;
+  int64_t n_src_frames;
+  int32_t n_frames;
+  int32_t first_frame;
+};
+cudaError_t launch_select_i8(const SelectI8Args &a, const SelectHostList *host_list,
+                             cudaStream_t stream);
 
 // ----------------------------------------------------------- attention ----
 constexpr int kMaxSpans = 4;

@@ -1,4 +1,5 @@
-// Fused 3D RoPE + KV-cache append (memory-bound).
+// Fused 3D RoPE + KV-cache append (memory-bound), into a bf16 cache or an
+// INT8 cache (codes + per-(token, head) scales).
 //
 // "Hy-Nomas: an 8.6B world model whose memory is a KV cache"
 // (ai.thesatyajit.com): section "How one segment is made", item "The blocks"
@@ -46,15 +47,54 @@ __device__ __forceinline__ uint4 rot_chunk(uint4 v, const float (&c)[4], const f
   return v;
 }
 
+// Symmetric INT8 quantisation of one (token, head): the 16 threads of the row
+// each hold 8 of the 128 bf16 values; the absmax is reduced with shuffles
+// inside the row's 16 lanes.  scale = absmax / 127 and code = rint(x / scale)
+// use round-to-nearest float32 division and round-half-even conversion, so
+// the codes are reproducible bit for bit; an all-zero head gets scale 0.
+__device__ __forceinline__ uint2 quant_chunk(uint4 v, unsigned row_mask, float *scale_out) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float x[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(row_mask, amax, off));
+  const float scale = __fdiv_rn(amax, 127.f);
+  uint32_t lo = 0, hi = 0;
+  if (scale > 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int q = __float2int_rn(__fdiv_rn(x[i], scale));
+      q = max(-127, min(127, q));
+      const uint32_t b = (uint32_t)(q & 0xff);
+      if (i < 4)
+        lo |= b << (8 * i);
+      else
+        hi |= b << (8 * (i - 4));
+    }
+  }
+  *scale_out = scale;
+  return make_uint2(lo, hi);
+}
+
+template <bool kQuant>
 __global__ void __launch_bounds__(kThreads)
 rope_append_kernel(const __grid_constant__ RopeArgs a) {
   const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 4);
   const int cc = threadIdx.x & 15;  // 16-byte chunk inside a head: dims 8cc..8cc+7
+  // The 16 lanes of this row (shuffle partners of the INT8 absmax).
+  const unsigned row_mask = 0xffffu << (threadIdx.x & 16);
 
   const bool do_q = a.q_in != nullptr && row < a.n_q_rows;
   const bool do_k = a.k_in != nullptr && row < a.n_kv_rows;
   const bool do_v = a.v_in != nullptr && row < a.n_kv_rows;
-  if (!do_q && !do_k && !do_v) return;
+  if (!do_q && !do_k && !do_v) return;  // uniform over the row's 16 lanes
 
   const bool rotate = row < a.n_video;
   float c[4] = {1.f, 1.f, 1.f, 1.f}, s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -97,8 +137,25 @@ rope_append_kernel(const __grid_constant__ RopeArgs a) {
     for (int g = 0; g < kHeadGroup; ++g) {
       const int64_t off = base + (int64_t)(h0 + g) * 16;
       if (do_q) q_out[off] = rotate ? rot_chunk(qv[g], c, s) : qv[g];
-      if (do_k) k_out[off] = rotate ? rot_chunk(kv[g], c, s) : kv[g];
-      if (do_v) v_out[off] = vv[g];
+      if constexpr (kQuant) {
+        // codes: 8 bytes per thread at [row][head][8cc..8cc+7]; one scale per (row, head)
+        const int64_t coff = row * (kRowElems / 8) + (int64_t)(h0 + g) * 16 + cc;
+        const int64_t soff = row * kHeads + h0 + g;
+        float sc;
+        if (do_k) {
+          const uint2 q8 = quant_chunk(rotate ? rot_chunk(kv[g], c, s) : kv[g], row_mask, &sc);
+          reinterpret_cast<uint2 *>(a.k_codes)[coff] = q8;
+          if (cc == 0) a.k_scales[soff] = sc;
+        }
+        if (do_v) {
+          const uint2 q8 = quant_chunk(vv[g], row_mask, &sc);
+          reinterpret_cast<uint2 *>(a.v_codes)[coff] = q8;
+          if (cc == 0) a.v_scales[soff] = sc;
+        }
+      } else {
+        if (do_k) k_out[off] = rotate ? rot_chunk(kv[g], c, s) : kv[g];
+        if (do_v) v_out[off] = vv[g];
+      }
     }
   }
 }
@@ -110,7 +167,16 @@ cudaError_t launch_rope_append(const RopeArgs &a, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   const int64_t blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
   if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  rope_append_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+  rope_append_kernel<false><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_append_i8(const RopeArgs &a, cudaStream_t stream) {
+  const int64_t rows = a.n_q_rows > a.n_kv_rows ? a.n_q_rows : a.n_kv_rows;
+  if (rows <= 0) return cudaSuccess;
+  const int64_t blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+  rope_append_kernel<true><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -199,3 +199,30 @@ def test_binding_fails_loudly_without_library(tmp_path):
             nm.load_library(str(tmp_path / "missing.so"))
     finally:
         nm._lib = saved
+
+
+def _cache_i8(capacity, length, tpf=24, base=FAKE):
+    return nm._KVCacheI8(base, base + capacity * 2048, base + 2 * capacity * 2048,
+                         base + 2 * capacity * 2048 + capacity * 64, capacity, length, tpf, 16, 128)
+
+
+def test_int8_append_and_select_validation(lib):
+    seg = FAKE + 10 ** 9
+    c = _cache_i8(100, 60)
+    st = lib.nomas_kvcache_append_i8(ctypes.byref(c), seg, seg + 48 * ROW, 48, None, None,
+                                     ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_CAPACITY and c.len == 60
+    bad = _cache_i8(100, 0)
+    bad.k_scale = None
+    st = lib.nomas_kvcache_append_i8(ctypes.byref(bad), seg, seg + 48 * ROW, 48, None, None,
+                                     ctypes.byref(_layout()), ctypes.byref(_cfg()), None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    src = _cache_i8(240, 240)
+    win = _cache(96, 0, tpf=0, base=FAKE + 10 ** 9)
+    idx = (ctypes.c_int32 * 2)(0, 10)
+    st = lib.nomas_kvcache_select_i8(ctypes.byref(src), idx, 2, 0, ctypes.byref(win), None, None)
+    assert st == nm.NOMAS_ERR_INDEX
+    overl = _cache(96, 0, tpf=0, base=FAKE + 2 * 240 * 2048)  # lands on the scales
+    ok_idx = (ctypes.c_int32 * 2)(0, 1)
+    st = lib.nomas_kvcache_select_i8(ctypes.byref(src), ok_idx, 2, 0, ctypes.byref(overl), None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
