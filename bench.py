@@ -39,7 +39,11 @@ def parse_args():
     p.add_argument("--steps", type=int, default=40)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["nomas", "reference"], default="nomas")
-    p.add_argument("--workload", choices=["720p", "bounded", "short", "mid", "tiny"], default="720p")
+    p.add_argument("--workload", choices=["720p", "bounded", "short", "mid", "tiny", "sweep"],
+                   default="720p")
+    p.add_argument("--int8", action="store_true",
+                   help="bounded workload with an INT8 history cache (quantising append, "
+                        "dequantising gather)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -184,9 +188,153 @@ class LayerStep:
             t.empty_like(self.o, device="cpu").pin_memory()
 
 
-def cpu_oracle_rate(step: LayerStep, budget_s: float, rows_per_chunk: int, max_rows: int):
-    """Times the fp64 oracle (RoPE of the sampled rows + their attention over
-    every key) on host cores; returns (TFLOP/s, rows, seconds, threads)."""
+class LayerStepI8:
+    """Bounded-history layer-step with an INT8 history cache.
+
+    Per step: 3D RoPE of the segment's Q and K into bf16 buffers, the rotated
+    K and V quantised into the INT8 cache, the frame list gathered back to a
+    bf16 window, then attention over window + text + segment.
+    """
+
+    def __init__(self, wname: str, seed: int):
+        import torch
+
+        import kv_cached_segment_b200 as nm
+        from seeded_inputs import WORKLOADS, bounded_frame_list, randn_bf16
+
+        self.nm, self.torch = nm, torch
+        w = self.w = WORKLOADS[wname]
+        if not w.select_frames:
+            raise SystemExit("--int8 needs the bounded workload")
+        dev = "cuda"
+        ns, nt = w.n_seg, w.n_text
+        self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        self.cache = nm.KVCacheI8.empty(w.n_cache + ns, w.tokens_per_frame)
+        chunk = 4 * w.tokens_per_frame * 30  # quantise the history in pieces
+        for r0 in range(0, w.n_cache, chunk):
+            r1 = min(w.n_cache, r0 + chunk)
+            hk = randn_bf16((r1 - r0, 16, 128), seed * 16 + 4 + r0, dev)
+            hv = randn_bf16((r1 - r0, 16, 128), seed * 16 + 5 + r0, dev)
+            nm.kvcache_append_i8(self.cache, hk, hv)
+        self.q = randn_bf16((w.n_q, 16, 128), seed * 16 + 1, dev)
+        self.k = randn_bf16((w.n_q, 16, 128), seed * 16 + 2, dev)
+        self.v = randn_bf16((w.n_q, 16, 128), seed * 16 + 3, dev)
+        self.q_rot = torch.empty_like(self.q)
+        self.k_rot = torch.empty_like(self.k)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.frames = bounded_frame_list(w, seed).tolist()
+        self.window = nm.KVCache.empty(w.n_window, 0)
+        self.launches_per_step = 4
+
+    def flops(self) -> float:
+        return self.w.attention_flops()
+
+    def run(self, ev=None):
+        nm, w = self.nm, self.w
+        ns = w.n_seg
+        self.cache.len = w.n_cache
+        nm.rope3d_qk(self.q, self.k, self.q_rot, self.k_rot, self.layout, self.cfg)
+        nm.kvcache_append_i8(self.cache, self.k_rot[:ns], self.v[:ns])
+        nm.kvcache_select(self.cache, self.frames, self.window)
+        spans = [self.window.span(), (self.k_rot[ns:], self.v[ns:]),
+                 (self.k_rot[:ns], self.v[:ns])]
+        if ev is not None:
+            ev[0].record()
+        nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
+        if ev is not None:
+            ev[1].record()
+
+    def host_inputs(self):
+        t = self.torch
+        return {n: getattr(self, n).cpu().pin_memory() for n in ("q", "k", "v")}, \
+            t.empty_like(self.o, device="cpu").pin_memory()
+
+
+class SweepStep:
+    """One denoising step of a whole segment: 54 layers of the 720p layer-step.
+
+    Every layer has its own resident cache of 55,200 tokens plus 512 text
+    tokens; each step uses fresh seeded Q and segment K/V (one set per
+    denoising step, 8 sets).  Per layer: 3D RoPE of Q and the segment K into
+    bf16 buffers, then attention over cache + text + segment.
+    """
+
+    def __init__(self, seed: int):
+        import torch
+
+        import kv_cached_segment_b200 as nm
+        from seeded_inputs import SWEEP_LAYERS, SWEEP_STEPS, WORKLOADS, randn_bf16
+
+        self.nm, self.torch = nm, torch
+        w = self.w = WORKLOADS["720p"]
+        dev = "cuda"
+        ns, nt = w.n_seg, w.n_text
+        self.layers, self.steps_per_segment = SWEEP_LAYERS, SWEEP_STEPS
+        self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        self.cache = []
+        for l in range(self.layers):
+            k = randn_bf16((w.n_cache + nt, 16, 128), seed * 1000 + 2 * l, dev)
+            v = randn_bf16((w.n_cache + nt, 16, 128), seed * 1000 + 2 * l + 1, dev)
+            self.cache.append((k, v))
+        self.inputs = [tuple(randn_bf16((w.n_q if i == 0 else ns, 16, 128),
+                                        seed * 100000 + 3 * s + i, dev) for i in range(3))
+                       for s in range(self.steps_per_segment)]
+        self.q_rot = torch.empty((w.n_q, 16, 128), dtype=torch.bfloat16, device=dev)
+        self.k_rot = torch.empty((ns, 16, 128), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty_like(self.q_rot)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.i = 0
+        self.launches_per_step = 3 * self.layers
+
+    def flops(self) -> float:
+        return self.w.attention_flops() * self.layers
+
+    def run(self, ev=None):
+        nm, w = self.nm, self.w
+        ns, nt = w.n_seg, w.n_text
+        q, k, v = self.inputs[self.i % self.steps_per_segment]
+        self.i += 1
+        # text rows of Q are copied by the RoPE pass; text K/V live with each layer
+        lay_q = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        lay_k = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, 0)
+        if ev is not None:
+            ev[0].record()
+        for l in range(self.layers):
+            ck, cv = self.cache[l]
+            nm.rope3d_qk(q, None, self.q_rot, None, lay_q, self.cfg)
+            nm.rope3d_qk(k, None, self.k_rot, None, lay_k, self.cfg)
+            spans = [(ck[:w.n_cache], cv[:w.n_cache]), (ck[w.n_cache:], cv[w.n_cache:]),
+                     (self.k_rot, v)]
+            nm.segment_attention(self.q_rot, spans, o=self.o, dev_err=self.err)
+        if ev is not None:
+            ev[1].record()
+
+    def host_inputs(self):
+        raise NotImplementedError
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise max of per-rank floats over all ranks (identity at world 1)."""
+    if world <= 1:
+        return [float(x) for x in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
+    """Times the fp64 oracle (RoPE of sampled query rows + their attention over
+    every key of the workload) on host cores; returns (TFLOP/s, rows, s, threads).
+
+    The oracle works from the seeded inputs (host copies of the resident
+    cache, the frame list and the segment), never from kernel outputs."""
     import numpy as np
     import torch
 
@@ -198,11 +346,13 @@ def cpu_oracle_rate(step: LayerStep, budget_s: float, rows_per_chunk: int, max_r
 
     w = step.w
     ns = w.n_seg
-    hist_k = step.window.k[:w.n_window] if step.frames else step.cache.k[:w.n_cache]
-    hist_v = step.window.v[:w.n_window] if step.frames else step.cache.v[:w.n_cache]
-    spans = [(f64(hist_k), f64(hist_v)), (f64(step.k[ns:]), f64(step.v[ns:])),
-             (f64(step.k[:ns]), f64(step.v[:ns]))]
+    hist_k, hist_v = f64(step.cache.k[:w.n_cache]), f64(step.cache.v[:w.n_cache])
+    if w.select_frames:
+        hist_k = oracle.kvcache_select(hist_k, step.frames, w.tokens_per_frame)
+        hist_v = oracle.kvcache_select(hist_v, step.frames, w.tokens_per_frame)
     t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    spans = [(hist_k, hist_v), (f64(step.k[ns:]), f64(step.v[ns:])),
+             (oracle.rope3d(f64(step.k[:ns]), ns, t, h, ww), f64(step.v[:ns]))]
     q_all = step.q
     rng = np.random.default_rng(0)
     done, elapsed = 0, 0.0
@@ -211,20 +361,39 @@ def cpu_oracle_rate(step: LayerStep, budget_s: float, rows_per_chunk: int, max_r
         rows = np.sort(rng.integers(0, ns, rows_per_chunk))
         q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
                                ww[rows])
-        k_seg = spans[2][0]
-        if done == 0:
-            k_seg = oracle.rope3d(k_seg, ns, t, h, ww)  # the segment's keys, once
-            spans[2] = (k_seg, spans[2][1])
         oracle.attention(q_rows, spans)
         done += rows.size
         elapsed = time.perf_counter() - t0
     flops = 4.0 * done * w.n_k * 128 * 16
+    return flops / elapsed / 1e12, done, elapsed, blas_threads()
+
+
+def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
-        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
     except Exception:  # noqa: BLE001
-        threads = os.cpu_count()
-    return flops / elapsed / 1e12, done, elapsed, threads
+        return os.cpu_count() or 1
+
+
+def make_step(args, rank):
+    if args.workload == "sweep":
+        return SweepStep(seed=1 + rank)
+    if args.int8:
+        return LayerStepI8(args.workload, seed=1 + rank)
+    return LayerStep(args.workload, seed=1 + rank)
+
+
+def workload_text(args, step) -> str:
+    w = step.w
+    if args.workload == "sweep":
+        return (f"sweep: {step.layers} layers x one denoising step of the 720p layer-step "
+                f"({w.frames}x{w.grid_h}x{w.grid_w} segment + {w.n_text} text over "
+                f"{w.n_cache} cached tokens per layer)")
+    hist = w.n_window if w.select_frames else w.n_cache
+    extra = " (INT8 history cache)" if args.int8 else ""
+    return (f"{w.name}: {w.frames}x{w.grid_h}x{w.grid_w} segment tokens + {w.n_text} text "
+            f"over {hist} history tokens{extra}")
 
 
 def main():
@@ -250,10 +419,11 @@ def main():
             dist.barrier()
 
     peaks, peak_src = load_peaks()
-    step = LayerStep(args.workload, seed=1 + rank)
+    step = make_step(args, rank)
     torch.cuda.synchronize()
 
-    for _ in range(max(3, args.warmup)):
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
         step.run()
     torch.cuda.synchronize()
     if int(step.err.item()) != 0:
@@ -280,13 +450,12 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop() if sampler else None
+    if int(step.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(step.err.item())}")
 
-    ms = start.elapsed_time(stop)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    if world > 1:
-        t = torch.tensor([ms, attn_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, attn_ms = float(t[0]), float(t[1])
+    ms, attn_ms = max_over_ranks(
+        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for a, b in evs)],
+        world, "cuda")
     ms_per_step = ms / args.steps
     flops = step.flops()
     value = flops * args.steps * world / (ms / 1e3) / 1e12
@@ -294,7 +463,7 @@ def main():
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.workload != "sweep":
         host_in, host_o = step.host_inputs()
         for _ in range(2):
             run_e2e(step, host_in, host_o)
@@ -307,18 +476,14 @@ def main():
             run_e2e(step, host_in, host_o)
         e1.record()
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
+        (e_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, "cuda")
         h2d = sum(x.numel() * x.element_size() for x in host_in.values())
         e2e = {"value": flops * n_e2e * world / (e_ms / 1e3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": host_o.numel() * 2,
                "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "sweep":
         rate, rows, secs, threads = cpu_oracle_rate(step, budget_s=12.0, rows_per_chunk=16,
                                                     max_rows=512)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -332,36 +497,41 @@ def main():
 
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     w = step.w
+    attn_per_step = getattr(step, "layers", 1)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": f"{w.name}: {w.frames}x{w.grid_h}x{w.grid_w} segment tokens + {w.n_text} "
-                        f"text over {w.n_window if w.select_frames else w.n_cache} history tokens",
+            "workload": workload_text(args, step),
             "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
             "attention_flops_per_step": flops,
-            "step": "fused rope3d+append" + (" + select" if w.select_frames else "")
-                    + " + segment attention",
+            "step": ("per layer: rope3d_qk x2 + segment attention" if args.workload == "sweep"
+                     else "rope3d_qk + int8 append + int8 select + segment attention" if args.int8
+                     else "fused rope3d+append" + (" + select" if w.select_frames else "")
+                     + " + segment attention"),
             "l2": "inputs larger than L2: each step reads "
-                  f"{(w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
+                  f"{attn_per_step * (w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
             "parallelism": f"independent layer-step per GPU x{world}",
         },
         "pct_of_measured_bf16_peak": 100.0 * value / peak,
         "pct_of_datasheet_bf16_peak": 100.0 * value / DATASHEET_BF16_TFLOPS,
-        "attention_ms": attn_ms,
-        "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn_tflops,
-                     "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "peak_source": f"{peak_src} bf16 burst",
+        "attention_ms": attn_ms / attn_per_step,
+        "roofline": {"kernel": "attention_kernel", "bound": "tensor",
+                     "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 burst",
                      "traffic": recorded_traffic(args.workload)},
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if args.workload == "sweep":
+        out["ms_per_segment"] = ms_per_step * step.steps_per_segment
+        out["roofline"]["note"] = "per-step average over the 54 layers (rope3d_qk launches included)"
     print(json.dumps(out), flush=True)
 
 
-def run_e2e(step: LayerStep, host_in, host_o):
+def run_e2e(step, host_in, host_o):
     step.q.copy_(host_in["q"], non_blocking=True)
     step.k.copy_(host_in["k"], non_blocking=True)
     step.v.copy_(host_in["v"], non_blocking=True)
@@ -379,7 +549,7 @@ def run_reference(args, rank, world):
     import oracle
     from seeded_inputs import WORKLOADS, layer_inputs
 
-    w = WORKLOADS[args.workload]
+    w = WORKLOADS["720p" if args.workload == "sweep" else args.workload]
     inp = layer_inputs(w, seed=1)
 
     def f64(t):

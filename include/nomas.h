@@ -211,9 +211,10 @@ typedef struct {
 /*
  * nomas_kvcache_append into an INT8 cache: the rotated segment keys (rounded
  * to bf16, as the bf16 path would store them) and the values are quantised
- * per (token, head) with scale = absmax / 127 and code = rint(x / scale),
- * both divisions rounded to nearest in fp32 and rint rounding half to even;
- * an all-zero (token, head) gets scale 0 and codes 0.  Q is handled exactly as
+ * per (token, head): a = absmax, stored scale = a / 127, code =
+ * rint(x * (127 / a)), divisions and product rounded to nearest in fp32 and
+ * rint rounding half to even; an all-zero (token, head) gets scale 0 and
+ * codes 0.  Q is handled exactly as
  * in nomas_kvcache_append.  Same errors as nomas_kvcache_append.
  */
 nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,

@@ -48,10 +48,11 @@ __device__ __forceinline__ uint4 rot_chunk(uint4 v, const float (&c)[4], const f
 }
 
 // Symmetric INT8 quantisation of one (token, head): the 16 threads of the row
-// each hold 8 of the 128 bf16 values; the absmax is reduced with shuffles
-// inside the row's 16 lanes.  scale = absmax / 127 and code = rint(x / scale)
-// use round-to-nearest float32 division and round-half-even conversion, so
-// the codes are reproducible bit for bit; an all-zero head gets scale 0.
+// each hold 8 of the 128 bf16 values; the absmax a is reduced with shuffles
+// inside the row's 16 lanes.  The stored scale is a / 127 and code =
+// rint(x * (127 / a)); the two divisions (one per token and head) and the
+// product round to nearest in float32 and the conversion rounds half to even,
+// so the codes are reproducible bit for bit; an all-zero head gets scale 0.
 __device__ __forceinline__ uint2 quant_chunk(uint4 v, unsigned row_mask, float *scale_out) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float x[8];
@@ -67,10 +68,11 @@ __device__ __forceinline__ uint2 quant_chunk(uint4 v, unsigned row_mask, float *
   for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(row_mask, amax, off));
   const float scale = __fdiv_rn(amax, 127.f);
   uint32_t lo = 0, hi = 0;
-  if (scale > 0.f) {
+  if (amax > 0.f) {
+    const float inv = __fdiv_rn(127.f, amax);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      int q = __float2int_rn(__fdiv_rn(x[i], scale));
+      int q = __float2int_rn(__fmul_rn(x[i], inv));
       q = max(-127, min(127, q));
       const uint32_t b = (uint32_t)(q & 0xff);
       if (i < 4)

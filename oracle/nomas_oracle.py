@@ -239,18 +239,21 @@ def quantize_int8(x_bits):
     [KV] "The 4090 preset": the cache is quantised once per segment to one
     byte per value plus an FP32 scale per token and head (4,224 B per token
     per layer for K and V together).  Reading (the page gives no formula):
-    absmax scaling in float32, scale = max_d |x_d| / 127 and code =
-    rint(x_d / scale), both divisions rounded to nearest in float32 and rint
-    rounding half to even; an all-zero (token, head) gets scale 0 and codes 0.
+    absmax scaling decided in float32: a = max_d |x_d|, scale = a / 127 (the
+    stored scale) and code = rint(x_d * (127 / a)), each division and the
+    product rounded to nearest in float32 and rint rounding half to even; an
+    all-zero (token, head) gets scale 0 and codes 0.
     Returns int8 codes [N][H][D] and float32 scales [N][H].
     """
     x = bf16_bits_to_f64(x_bits).astype(np.float32)          # exact
     amax = np.max(np.abs(x), axis=2)                           # exact
     scale = (amax / np.float32(127.0)).astype(np.float32)      # fp32 RN
-    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
-    q = (x / safe[:, :, None]).astype(np.float32)              # fp32 RN
+    zero = amax == 0
+    safe = np.where(zero, np.float32(1.0), amax).astype(np.float32)
+    inv = (np.float32(127.0) / safe).astype(np.float32)        # fp32 RN
+    q = (x * inv[:, :, None]).astype(np.float32)               # fp32 RN
     codes = np.clip(np.rint(q), -127, 127).astype(np.int8)
-    codes[scale == 0] = 0
+    codes[zero] = 0
     return codes, scale
 
 
