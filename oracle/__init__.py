@@ -24,4 +24,6 @@ from .nomas_oracle import (  # noqa: F401
     f32_to_bf16_bits,
     quantize_int8,
     dequantize_int8,
+    key_tiles,
+    block_sparse_attention,
 )

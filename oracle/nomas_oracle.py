@@ -262,3 +262,53 @@ def dequantize_int8(codes, scales) -> np.ndarray:
     prod = (np.asarray(codes, dtype=np.float32) *
             np.asarray(scales, dtype=np.float32)[:, :, None]).astype(np.float32)
     return f32_to_bf16_bits(prod)
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse segment attention
+# ---------------------------------------------------------------------------
+def key_tiles(span_lens, block_k: int = 128):
+    """Key tiles of the concatenated spans: (span, first key, end key) each.
+
+    Tiles never straddle spans: span s contributes ceil(len_s / block_k) tiles,
+    the last one short.  A tile's global id is its index in this list.
+    """
+    tiles = []
+    for s, n in enumerate(span_lens):
+        for a in range(0, int(n), block_k):
+            tiles.append((s, a, min(int(n), a + block_k)))
+    return tiles
+
+
+def block_sparse_attention(q, spans, tile_lists, block_q: int = 256, block_k: int = 128,
+                           scale=None):
+    """Attention where each (query block, head) sees only listed key tiles.
+
+    [IT]/[4090] single-GPU preset: block-sparse attention keeps a fraction of
+    the candidate video key blocks after the first denoising steps; the pages
+    do not state the selection rule, so the selection is an input here:
+    ``tile_lists[b][h]`` lists the global tile ids (see ``key_tiles``) that
+    query rows [b * block_q, (b + 1) * block_q) of head h attend to.  Within
+    that key set the result is the plain softmax attention of
+    ``attention_rows``.  Each listed tile contributes its keys once per
+    listing; ids outside the tile list are ignored; an empty set gives O = 0
+    and LSE = -inf.
+    """
+    nq, n_heads, d = q.shape
+    tiles = key_tiles([s[0].shape[0] for s in spans], block_k)
+    out = np.zeros((nq, n_heads, d), dtype=np.float64)
+    lse = np.full((n_heads, nq), -np.inf, dtype=np.float64)
+    for b in range(len(tile_lists)):
+        rows = np.arange(b * block_q, min(nq, (b + 1) * block_q))
+        if rows.size == 0:
+            continue
+        for h in range(n_heads):
+            sel = [tiles[g] for g in tile_lists[b][h] if 0 <= g < len(tiles)]
+            if not sel:
+                continue
+            kh = np.concatenate([spans[s][0][a:e, h:h + 1] for s, a, e in sel])
+            vh = np.concatenate([spans[s][1][a:e, h:h + 1] for s, a, e in sel])
+            o_h, l_h = attention_rows(q[:, h:h + 1], rows, [(kh, vh)], scale)
+            out[rows, h] = o_h[:, 0]
+            lse[h, rows] = l_h[0]
+    return out, lse

@@ -406,3 +406,42 @@ def test_int8_zero_rows():
     codes, scales = O.quantize_int8(z)
     assert np.all(codes == 0) and np.all(scales == 0)
     assert np.all(O.dequantize_int8(codes, scales) == 0)
+
+
+# ------------------------------------------------------- block-sparse -----
+def test_key_tiles_never_straddle_spans():
+    t = O.key_tiles([300, 0, 128, 5], 128)
+    assert t == [(0, 0, 128), (0, 128, 256), (0, 256, 300), (2, 0, 128), (3, 0, 5)]
+
+
+def test_block_sparse_with_every_tile_is_dense():
+    r = rng(30)
+    q = r.standard_normal((300, 2, 16))
+    spans = [(r.standard_normal((n, 2, 16)), r.standard_normal((n, 2, 16))) for n in (130, 7)]
+    n_tiles = len(O.key_tiles([130, 7], 128))
+    lists = [[list(range(n_tiles))] * 2 for _ in range(2)]
+    o, l = O.block_sparse_attention(q, spans, lists)
+    o2, l2 = O.attention(q, spans)
+    assert np.allclose(o, o2, atol=1e-12) and np.allclose(l, l2, atol=1e-12)
+
+
+def test_block_sparse_one_tile_brute_force():
+    r = rng(31)
+    q = r.standard_normal((5, 1, 8))
+    k = r.standard_normal((12, 1, 8))
+    v = r.standard_normal((12, 1, 8))
+    # tiles of 4 keys: keep tile 2 (keys 8..11) only; ids 7 and -1 are ignored
+    o, l = O.block_sparse_attention(q, [(k, v)], [[[2, 7, -1]]], block_q=8, block_k=4)
+    ob, lb = brute_force_attention(q, k[8:12], v[8:12], 1 / math.sqrt(8))
+    assert np.allclose(o, ob, atol=1e-12) and np.allclose(l, lb, atol=1e-12)
+
+
+def test_block_sparse_blocks_are_independent_and_empty_gives_zero():
+    r = rng(32)
+    q = r.standard_normal((10, 1, 8))
+    k = r.standard_normal((8, 1, 8))
+    v = r.standard_normal((8, 1, 8))
+    o, l = O.block_sparse_attention(q, [(k, v)], [[[0]], [[]]], block_q=5, block_k=4)
+    o_a, l_a = O.attention(q[:5], [(k[:4], v[:4])])
+    assert np.allclose(o[:5], o_a, atol=1e-13) and np.allclose(l[:, :5], l_a, atol=1e-13)
+    assert np.all(o[5:] == 0) and np.all(np.isneginf(l[:, 5:]))
