@@ -24,6 +24,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -44,6 +46,9 @@ def parse_args():
     p.add_argument("--int8", action="store_true",
                    help="bounded workload with an INT8 history cache (quantising append, "
                         "dequantising gather)")
+    p.add_argument("--sparse", type=float, default=0.0,
+                   help="block-sparse attention keeping this fraction of the video key tiles "
+                        "(text tiles always kept); 0 = dense")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -159,9 +164,31 @@ class LayerStep:
         else:
             self.frames = None
         self.launches_per_step = 3 if self.frames else 2
+        self.sparse = None
+
+    def use_sparse(self, fraction: float, seed: int):
+        """Seeded block-sparse selection: text tiles kept, `fraction` of the
+        history and segment tiles per (query block, head)."""
+        from seeded_inputs import sparse_tile_lists
+
+        w, torch = self.w, self.torch
+        hist = w.n_window if w.select_frames else w.n_cache
+        lens = [hist, w.n_text, w.n_seg]
+        lists, counts = sparse_tile_lists(w.n_q, lens, keep_spans=[1], candidate_spans=[0, 2],
+                                          fraction=fraction, seed=seed)
+        # keys actually attended: every listed tile is full except span ends
+        tile_keys = []
+        for n in lens:
+            tile_keys += [min(128, n - a) for a in range(0, n, 128)]
+        tile_keys = np.asarray(tile_keys)
+        rows = np.minimum(256, w.n_q - 256 * np.arange(lists.shape[0]))
+        keys = np.array([[tile_keys[lists[b, h, :counts[b, h]]].sum() for h in range(16)]
+                         for b in range(lists.shape[0])])
+        self.sparse_flops = float(4.0 * 128 * (rows[:, None] * keys).sum())
+        self.sparse = (torch.from_numpy(lists).cuda(), torch.from_numpy(counts).cuda())
 
     def flops(self) -> float:
-        return self.w.attention_flops()
+        return self.sparse_flops if self.sparse is not None else self.w.attention_flops()
 
     def run(self, ev=None):
         nm, w = self.nm, self.w
@@ -177,7 +204,11 @@ class LayerStep:
         spans = [hist, (self.k[ns:], self.v[ns:]), self.cache.span(w.n_cache, w.n_cache + ns)]
         if ev is not None:
             ev[0].record()
-        nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
+        if self.sparse is not None:
+            nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=self.o, lse=self.lse,
+                                        dev_err=self.err)
+        else:
+            nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
         if ev is not None:
             ev[1].record()
 
@@ -381,7 +412,10 @@ def make_step(args, rank):
         return SweepStep(seed=1 + rank)
     if args.int8:
         return LayerStepI8(args.workload, seed=1 + rank)
-    return LayerStep(args.workload, seed=1 + rank)
+    step = LayerStep(args.workload, seed=1 + rank)
+    if args.sparse > 0:
+        step.use_sparse(args.sparse, seed=1 + rank)
+    return step
 
 
 def workload_text(args, step) -> str:
@@ -392,6 +426,9 @@ def workload_text(args, step) -> str:
                 f"{w.n_cache} cached tokens per layer)")
     hist = w.n_window if w.select_frames else w.n_cache
     extra = " (INT8 history cache)" if args.int8 else ""
+    if args.sparse > 0:
+        extra += (f" (block-sparse: text kept, {100 * args.sparse:.0f}% of video key tiles "
+                  f"per 256-query block and head)")
     return (f"{w.name}: {w.frames}x{w.grid_h}x{w.grid_w} segment tokens + {w.n_text} text "
             f"over {hist} history tokens{extra}")
 

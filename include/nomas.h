@@ -50,6 +50,7 @@ typedef enum {
 /* Bits ORed into *dev_err by kernels. */
 #define NOMAS_DEVERR_BAD_FRAME_INDEX 0x1 /* select: device list entry out of range */
 #define NOMAS_DEVERR_WAIT_TIMEOUT 0x2    /* attention: a pipeline wait timed out   */
+#define NOMAS_DEVERR_BAD_TILE_INDEX 0x4  /* sparse attention: tile id out of range */
 
 #define NOMAS_HEADS 16
 #define NOMAS_HEAD_DIM 128
@@ -271,6 +272,30 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
                                         int32_t n_spans, void *o, float *lse, float softmax_scale,
                                         int32_t heads, int32_t head_dim, int32_t *dev_err,
                                         const nomas_attention_opts *opts, void *stream);
+
+/*
+ * Block-sparse segment attention.  The single-GPU preset of the pages keeps
+ * only a fraction of the candidate video key blocks after the first denoising
+ * steps ("Hy-Nomas en una RTX 4090", section "El preset de una GPU": dense on the
+ * first two denoising steps, then 25% of the candidate video blocks); the pages do not
+ * give the selection rule, so the selection is an input.  Keys are cut into
+ * tiles of NOMAS_SPARSE_BLOCK_K keys per span (the last tile of a span is
+ * short), numbered consecutively over the spans in order; queries into blocks
+ * of NOMAS_SPARSE_BLOCK_Q rows.  Query block b of head h attends to exactly
+ * the tiles listed in tile_list[(b * heads + h) * max_tiles + i] for
+ * i < tile_count[b * heads + h] (device int32 arrays; a tile listed twice
+ * counts twice).  Ids outside the tiles are skipped and set
+ * NOMAS_DEVERR_BAD_TILE_INDEX in *dev_err (required).  A block with no valid
+ * tile gets O = 0, LSE = -inf.  Otherwise as nomas_segment_attention.
+ */
+#define NOMAS_SPARSE_BLOCK_Q 256
+#define NOMAS_SPARSE_BLOCK_K 128
+nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
+                                            const nomas_kv_span *spans, int32_t n_spans,
+                                            const int32_t *tile_list, const int32_t *tile_count,
+                                            int32_t max_tiles, void *o, float *lse,
+                                            float softmax_scale, int32_t heads, int32_t head_dim,
+                                            int32_t *dev_err, void *stream);
 
 #ifdef __cplusplus
 }

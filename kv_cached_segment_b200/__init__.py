@@ -43,7 +43,11 @@ EXPORTED_SYMBOLS = (
     "nomas_temporal_context_frames",
     "nomas_kvcache_append_i8",
     "nomas_kvcache_select_i8",
+    "nomas_segment_attention_sparse",
 )
+SPARSE_BLOCK_Q = 256
+SPARSE_BLOCK_K = 128
+DEVERR_BAD_TILE_INDEX = 0x4
 
 
 class NomasError(RuntimeError):
@@ -127,6 +131,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_kvcache_select_i8.restype = ctypes.c_int
     lib.nomas_kvcache_select_i8.argtypes = [ctypes.POINTER(_KVCacheI8), P, I32, I32,
                                             ctypes.POINTER(_KVCache), P, P]
+    lib.nomas_segment_attention_sparse.restype = ctypes.c_int
+    lib.nomas_segment_attention_sparse.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, I32,
+                                                   P, P, F32, I32, I32, P, P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -385,4 +392,41 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         _check(lib.nomas_segment_attention(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
                                            float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
                                            _stream(stream)))
+    return o
+
+
+def segment_attention_sparse(q, spans, tile_list, tile_count, o=None, lse=None,
+                             softmax_scale: float = 0.0, dev_err=None, stream=None):
+    """Block-sparse attention: query block b (256 rows) of head h attends to the
+    128-key tiles tile_list[b, h, :tile_count[b, h]] (tiles numbered over the
+    spans in order).  tile_list: CUDA int32 [blocks][16][max_tiles];
+    tile_count: CUDA int32 [blocks][16]; dev_err: CUDA int32 word (required)."""
+    lib = load_library()
+    n_q = _rows(q, "q")
+    if o is None:
+        o = torch.empty_like(q)
+    _rows(o, "o")
+    n_blocks = (n_q + SPARSE_BLOCK_Q - 1) // SPARSE_BLOCK_Q
+    for t, name in ((tile_list, "tile_list"), (tile_count, "tile_count")):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA int32 tensor")
+    if tile_list.dim() != 3 or tile_list.shape[:2] != (n_blocks, HEADS):
+        raise ValueError(f"tile_list must have shape [{n_blocks}][{HEADS}][max_tiles]")
+    if tuple(tile_count.shape) != (n_blocks, HEADS):
+        raise ValueError(f"tile_count must have shape [{n_blocks}][{HEADS}]")
+    if dev_err is None or dev_err.dtype != torch.int32 or not dev_err.is_cuda:
+        raise TypeError("dev_err must be a CUDA int32 tensor")
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_cuda or
+                            lse.numel() != HEADS * n_q or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous CUDA fp32 tensor of heads * n_q elements")
+    arr = (_KVSpan * max(1, len(spans)))()
+    for i, (k, v) in enumerate(spans):
+        nk = _rows(k, f"span {i} k")
+        if _rows(v, f"span {i} v") != nk:
+            raise ValueError(f"span {i}: k and v differ in rows")
+        arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
+    _check(lib.nomas_segment_attention_sparse(_ptr(q), n_q, arr, len(spans), tile_list.data_ptr(),
+                                              tile_count.data_ptr(), tile_list.shape[2], _ptr(o),
+                                              _ptr(lse), float(softmax_scale), HEADS, HEAD_DIM,
+                                              dev_err.data_ptr(), _stream(stream)))
     return o

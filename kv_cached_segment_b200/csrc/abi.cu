@@ -312,6 +312,12 @@ nomas_status select_common(const CacheView &src, int32_t tokens_per_frame,
 
 unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s per pipeline wait
 
+nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                              int32_t n_spans, const int32_t *tile_list,
+                              const int32_t *tile_count, int32_t max_tiles, void *o, float *lse,
+                              float softmax_scale, int32_t heads, int32_t head_dim,
+                              int32_t *dev_err, const nomas_attention_opts *opts, void *stream);
+
 }  // namespace
 
 extern "C" {
@@ -419,6 +425,36 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
                                         int32_t n_spans, void *o, float *lse, float softmax_scale,
                                         int32_t heads, int32_t head_dim, int32_t *dev_err,
                                         const nomas_attention_opts *opts, void *stream) {
+  return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
+                          heads, head_dim, dev_err, opts, stream);
+}
+
+nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
+                                            const nomas_kv_span *spans, int32_t n_spans,
+                                            const int32_t *tile_list, const int32_t *tile_count,
+                                            int32_t max_tiles, void *o, float *lse,
+                                            float softmax_scale, int32_t heads, int32_t head_dim,
+                                            int32_t *dev_err, void *stream) {
+  if (tile_list == nullptr || tile_count == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "tile_list and tile_count are required");
+  if (max_tiles < 0) return fail(NOMAS_ERR_INVALID_ARG, "max_tiles < 0");
+  if (dev_err == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "dev_err is required with a device-resident tile list");
+  if ((reinterpret_cast<uintptr_t>(tile_list) & 3u) || (reinterpret_cast<uintptr_t>(tile_count) & 3u))
+    return fail(NOMAS_ERR_INVALID_ARG, "tile_list and tile_count must be 4-byte aligned");
+  return attention_common(q, n_q, spans, n_spans, tile_list, tile_count, max_tiles, o, lse,
+                          softmax_scale, heads, head_dim, dev_err, nullptr, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                              int32_t n_spans, const int32_t *tile_list,
+                              const int32_t *tile_count, int32_t max_tiles, void *o, float *lse,
+                              float softmax_scale, int32_t heads, int32_t head_dim,
+                              int32_t *dev_err, const nomas_attention_opts *opts, void *stream) {
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   if (n_spans < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_spans < 0");
@@ -453,8 +489,12 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
     if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len)) != NOMAS_OK) return st;
     if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len)) != NOMAS_OK) return st;
     a.span_len[n_used] = sp.len;
+    a.tile_base[n_used + 1] = a.tile_base[n_used] + (int32_t)((sp.len + 127) / 128);
     ++n_used;
   }
+  a.tile_list = tile_list;
+  a.tile_count = tile_count;
+  a.max_tiles = max_tiles;
   if (n_used == 0) {
     const cudaError_t e = launch_attention_empty(static_cast<uint16_t *>(o), lse, n_q,
                                                  static_cast<cudaStream_t>(stream));
@@ -482,4 +522,5 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
   return ok();
 }
 
-}  // extern "C"
+}  // namespace
+

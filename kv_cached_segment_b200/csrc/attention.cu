@@ -347,6 +347,48 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
 
 __device__ __forceinline__ int num_tiles(int64_t len) { return (int)((len + kBN - 1) / kBN); }
 
+// Walks this block's key tiles as (span, tile within the span).  Dense mode
+// visits every tile of every span in order with two counters; sparse mode
+// reads the block's list of global tile ids (tiles numbered across the
+// concatenated spans) and skips ids outside the spans -- every role walks the
+// same list the same way, so they agree on the sequence.
+template <bool kSparse>
+struct TileWalk {
+  const AttnArgs &p;
+  const int32_t *list;
+  int n_list;
+  int idx = 0, s = 0, kt = 0;
+  __device__ TileWalk(const AttnArgs &a, const int32_t *l, int n) : p(a), list(l), n_list(n) {}
+  // Next tile; false at the end.  `bad` is set when an invalid id was skipped.
+  __device__ __forceinline__ bool next(int *span, int *ktile, bool *bad) {
+    if constexpr (kSparse) {
+      while (idx < n_list) {
+        const int g = list[idx++];
+        if (g < 0 || g >= p.tile_base[p.n_spans]) {
+          *bad = true;
+          continue;
+        }
+        int t = 0;
+        while (t + 1 < p.n_spans && g >= p.tile_base[t + 1]) ++t;
+        *span = t;
+        *ktile = g - p.tile_base[t];
+        return true;
+      }
+      return false;
+    } else {
+      while (s < p.n_spans && kt >= num_tiles(p.span_len[s])) {
+        ++s;
+        kt = 0;
+      }
+      if (s >= p.n_spans) return false;
+      *span = s;
+      *ktile = kt++;
+      return true;
+    }
+  }
+};
+
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_kernel(const __grid_constant__ AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
@@ -394,8 +436,20 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
   const uint32_t tmem_base = *tmem_slot;
 
   const WaitCtl ctl{abort_flag, p.dev_err, p.wait_limit_ns};
-  int n_kv = 0;
-  for (int s = 0; s < p.n_spans; ++s) n_kv += num_tiles(p.span_len[s]);
+  // This block's key tiles: the whole key sequence, or its sparse list.
+  const int32_t *list = nullptr;
+  int n_list = 0;
+  int n_kv = p.tile_base[p.n_spans];  // K/V tiles this block streams
+  if constexpr (kSparse) {
+    const int64_t row = (int64_t)blockIdx.x * kHeads + head;
+    list = p.tile_list + row * p.max_tiles;
+    n_list = min(max(p.tile_count[row], 0), p.max_tiles);
+    n_kv = 0;
+    TileWalk<true> w(p, list, n_list);
+    int s_, kt_;
+    bool bad_ = false;
+    while (w.next(&s_, &kt_, &bad_)) ++n_kv;
+  }
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -409,9 +463,11 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
                       head * kHeadDim + c * 64, q_row0 + i * kBM, pol_q);
       int t = 0;
       bool ok = true;
-      for (int s = 0; s < p.n_spans && ok; ++s) {
-        const int nt = num_tiles(p.span_len[s]);
-        for (int kt = 0; kt < nt && ok; ++kt) {
+      TileWalk<kSparse> walk(p, list, n_list);
+      int s, kt;
+      bool bad = false;
+      while (ok && walk.next(&s, &kt, &bad)) {
+        {
           for (int which = 0; which < 2; ++which, ++t) {
             // Testing hook: leave one load out so that a consumer wait runs
             // out of time (exercises the bounded-wait abort path).
@@ -430,6 +486,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           }
         }
       }
+      if (bad && p.dev_err != nullptr) atomicOr(p.dev_err, NOMAS_DEVERR_BAD_TILE_INDEX);
       // Teardown: wait until every load this lane issued has landed.
       drain_phase(bar(kBarQFull), 0, p.wait_limit_ns);
       for (int u = (t > kStages ? t - kStages : 0); u < t; ++u)
@@ -512,10 +569,12 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
     float l = 0.f;        // running row sum of exp2(...)
     bool ok = true;
     int j = 0;
-    for (int s = 0; s < p.n_spans && ok; ++s) {
+    TileWalk<kSparse> walk(p, list, n_list);
+    int s, kt;
+    bool bad = false;
+    while (ok && walk.next(&s, &kt, &bad)) {
       const int64_t len = p.span_len[s];
-      const int nt = num_tiles(len);
-      for (int kt = 0; kt < nt; ++kt, ++j) {
+      {
         // Warp-uniform outcome: the tcgen05 loads and stores below are
         // warp-collective, so a lane that saw the abort flag takes the whole
         // warp with it.
@@ -642,6 +701,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
         tmem::wait_st();
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + tile));
+        ++j;
       }
     }
     // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l).
@@ -672,6 +732,16 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       }
       if (p.lse != nullptr && row < p.n_q)
         p.lse[(int64_t)head * p.n_q + row] = (m + log2f(l)) * 0.69314718055994531f;
+    } else if (ok && n_kv == 0) {
+      // No key selected for this block (a sparse list with no valid entry):
+      // the empty sums give O = 0 and LSE = -inf.
+      const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
+      if (row < p.n_q) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.o + row * kRowElems + head * kHeadDim);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+        if (p.lse != nullptr) p.lse[(int64_t)head * p.n_q + row] = -INFINITY;
+      }
     }
   }
 
@@ -705,7 +775,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attention_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemAlloc);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -714,7 +787,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   if (q_blocks <= 0) return cudaSuccess;
   if (q_blocks > 0x7fffffff) return cudaErrorInvalidValue;
   dim3 grid((unsigned)q_blocks, kHeads);
-  attention_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a);
+  if (a.tile_list != nullptr)
+    attention_kernel<true><<<grid, kThreads, kSmemAlloc, stream>>>(a);
+  else
+    attention_kernel<false><<<grid, kThreads, kSmemAlloc, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -86,6 +86,11 @@ struct AttnArgs {
   int32_t *dev_err;            // may be null
   unsigned long long wait_limit_ns;
   int32_t testing_skip_load;   // -1, or the K/V load index the producer leaves out
+  // Block-sparse selection (null tile_list: every tile of every span, in order).
+  const int32_t *tile_list;    // [q_blocks][heads][max_tiles] global key-tile ids
+  const int32_t *tile_count;   // [q_blocks][heads] entries used in each row
+  int32_t max_tiles;
+  int32_t tile_base[kMaxSpans + 1];  // first global tile id of each span; [n_spans] = total
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,

@@ -284,9 +284,10 @@ def block_sparse_attention(q, spans, tile_lists, block_q: int = 256, block_k: in
                            scale=None):
     """Attention where each (query block, head) sees only listed key tiles.
 
-    [IT]/[4090] single-GPU preset: block-sparse attention keeps a fraction of
-    the candidate video key blocks after the first denoising steps; the pages
-    do not state the selection rule, so the selection is an input here:
+    [4090] "El preset de una GPU": the single-GPU preset's attention is dense
+    on the first two denoising steps and then keeps 25% of the candidate
+    video key blocks; the pages do not state the selection rule, so the
+    selection is an input here:
     ``tile_lists[b][h]`` lists the global tile ids (see ``key_tiles``) that
     query rows [b * block_q, (b + 1) * block_q) of head h attend to.  Within
     that key set the result is the plain softmax attention of

@@ -149,3 +149,35 @@ def random_frame_list(n_src_frames: int, n: int, seed: int) -> np.ndarray:
     """Uniform random frame indices in [0, n_src_frames), repeats allowed."""
     rng = np.random.default_rng(seed)
     return rng.integers(0, n_src_frames, size=n).astype(np.int32)
+
+
+def sparse_tile_lists(n_q: int, span_lens, keep_spans, candidate_spans, fraction: float,
+                      seed: int, heads: int = HEADS, block_q: int = 256, block_k: int = 128):
+    """Seeded block-sparse selection: per (query block, head), every key tile
+    of the spans in ``keep_spans`` plus a random ``fraction`` of the tiles of
+    ``candidate_spans``.  Returns (lists [blocks][heads][max] int32 padded
+    with -1, counts [blocks][heads] int32).  The pages give no selection
+    rule; this only produces inputs of the right shape and density."""
+    rng = np.random.default_rng(seed)
+    first, span_tiles = [], []
+    t = 0
+    for n in span_lens:
+        k = (int(n) + block_k - 1) // block_k
+        first.append(t)
+        span_tiles.append(k)
+        t += k
+    keep = [first[s] + i for s in keep_spans for i in range(span_tiles[s])]
+    cand = np.array([first[s] + i for s in candidate_spans for i in range(span_tiles[s])],
+                    dtype=np.int64)
+    n_pick = int(round(fraction * cand.size))
+    n_blocks = (n_q + block_q - 1) // block_q
+    max_tiles = len(keep) + n_pick
+    lists = np.full((n_blocks, heads, max(1, max_tiles)), -1, dtype=np.int32)
+    counts = np.zeros((n_blocks, heads), dtype=np.int32)
+    for b in range(n_blocks):
+        for h in range(heads):
+            pick = np.sort(rng.choice(cand, size=n_pick, replace=False)) if n_pick else []
+            sel = sorted(keep + [int(x) for x in pick])
+            lists[b, h, :len(sel)] = sel
+            counts[b, h] = len(sel)
+    return lists, counts
