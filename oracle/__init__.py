@@ -26,4 +26,5 @@ from .nomas_oracle import (  # noqa: F401
     dequantize_int8,
     key_tiles,
     block_sparse_attention,
+    merge_partials,
 )

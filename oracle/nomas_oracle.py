@@ -313,3 +313,30 @@ def block_sparse_attention(q, spans, tile_lists, block_q: int = 256, block_k: in
             out[rows, h] = o_h[:, 0]
             lse[h, rows] = l_h[0]
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Sharded keys: merging partial results
+# ---------------------------------------------------------------------------
+def merge_partials(o_parts, lse_parts):
+    """Combine attention results computed over disjoint key subsets.
+
+    [KV] "What 'world memory' stores" (the standard preset spreads the cache
+    over eight GPUs, sp_size 8): each GPU attends over its part of the keys.
+    With LSE_r = ln sum_{j in part r} e^{s_j} and O_r the softmax-weighted V
+    of part r, the whole is LSE = ln sum_r e^{LSE_r} and
+    O = sum_r e^{LSE_r - LSE} O_r (the sums over parts regroup the sums over
+    keys).  Parts with LSE = -inf (no keys) contribute nothing; if every part
+    is empty, O = 0 and LSE = -inf.
+    o_parts: [R][Nq][H][D], lse_parts: [R][H][Nq] (natural log).
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = lse_parts.max(axis=0)                                   # [H][Nq]
+    safe_m = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse_parts - safe_m[None])                        # [R][H][Nq]
+    total = w.sum(axis=0)
+    lse = np.where(total > 0, safe_m + np.log(np.where(total > 0, total, 1.0)), -np.inf)
+    wn = np.where(total[None] > 0, w / np.where(total > 0, total, 1.0)[None], 0.0)
+    out = np.einsum("rhq,rqhd->qhd", wn, o_parts)
+    return out, lse

@@ -445,3 +445,32 @@ def test_block_sparse_blocks_are_independent_and_empty_gives_zero():
     o_a, l_a = O.attention(q[:5], [(k[:4], v[:4])])
     assert np.allclose(o[:5], o_a, atol=1e-13) and np.allclose(l[:, :5], l_a, atol=1e-13)
     assert np.all(o[5:] == 0) and np.all(np.isneginf(l[:, 5:]))
+
+
+# ------------------------------------------------------- sharded merge -----
+def test_merge_two_equal_parts_is_the_average():
+    # Equal LSE in both parts: weights 1/2 each, LSE grows by ln 2.
+    o = np.stack([np.full((3, 1, 4), 2.0), np.full((3, 1, 4), 4.0)])
+    lse = np.full((2, 1, 3), 1.5)
+    out, l = O.merge_partials(o, lse)
+    assert np.allclose(out, 3.0) and np.allclose(l, 1.5 + math.log(2))
+
+
+def test_merge_ignores_empty_parts_and_all_empty_is_zero():
+    o = np.stack([np.ones((2, 1, 4)) * 5, np.ones((2, 1, 4)) * 9])
+    lse = np.array([[[0.25, -np.inf]], [[-np.inf, -np.inf]]])
+    out, l = O.merge_partials(o, lse)
+    assert np.allclose(out[0], 5.0) and l[0, 0] == 0.25
+    assert np.all(out[1] == 0) and np.isneginf(l[0, 1])
+
+
+def test_merge_of_shards_equals_whole():
+    r = rng(40)
+    q = r.standard_normal((7, 2, 16))
+    k = r.standard_normal((50, 2, 16))
+    v = r.standard_normal((50, 2, 16))
+    cuts = [0, 13, 13, 31, 50]   # includes an empty shard
+    parts = [O.attention(q, [(k[a:b], v[a:b])]) for a, b in zip(cuts[:-1], cuts[1:])]
+    out, l = O.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    o_all, l_all = O.attention(q, [(k, v)])
+    assert np.allclose(out, o_all, atol=1e-12) and np.allclose(l, l_all, atol=1e-12)
