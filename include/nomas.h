@@ -297,6 +297,22 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
                                             float softmax_scale, int32_t heads, int32_t head_dim,
                                             int32_t *dev_err, void *stream);
 
+/*
+ * Merge of attention results over disjoint key shards ("What 'world memory'
+ * stores": the standard preset spreads the cache over eight GPUs, sp_size 8;
+ * each GPU attends over its shard and the partial results are combined):
+ * LSE = ln sum_r e^{LSE_r}, O = sum_r e^{LSE_r - LSE} O_r, accumulated in fp32.
+ *   o_parts  : [n_parts][n_q][heads][head_dim] bf16 partial outputs (device).
+ *   lse_parts: [n_parts][heads][n_q] fp32 partial LSEs (natural log, device).
+ *   o        : [n_q][heads][head_dim] bf16 output; lse: optional [heads][n_q].
+ * Parts with LSE = -inf are empty and contribute nothing; if all are empty the
+ * row gets O = 0 and LSE = -inf.  Outputs must not overlap the inputs.
+ * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,
+                                   int64_t n_q, void *o, float *lse, int32_t heads,
+                                   int32_t head_dim, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

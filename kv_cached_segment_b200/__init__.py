@@ -44,6 +44,7 @@ EXPORTED_SYMBOLS = (
     "nomas_kvcache_append_i8",
     "nomas_kvcache_select_i8",
     "nomas_segment_attention_sparse",
+    "nomas_attention_merge",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -134,6 +135,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_segment_attention_sparse.restype = ctypes.c_int
     lib.nomas_segment_attention_sparse.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, I32,
                                                    P, P, F32, I32, I32, P, P]
+    lib.nomas_attention_merge.restype = ctypes.c_int
+    lib.nomas_attention_merge.argtypes = [P, P, I32, I64, P, P, I32, I32, P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -430,3 +433,54 @@ def segment_attention_sparse(q, spans, tile_list, tile_count, o=None, lse=None,
                                               _ptr(lse), float(softmax_scale), HEADS, HEAD_DIM,
                                               dev_err.data_ptr(), _stream(stream)))
     return o
+
+
+def attention_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
+    """Combine partial results over disjoint key shards.
+
+    o_parts: CUDA bf16 [R][n_q][16][128]; lse_parts: CUDA fp32 [R][16][n_q].
+    Returns o ([n_q][16][128] bf16); fills lse ([16][n_q] fp32) if given."""
+    lib = load_library()
+    if o_parts.dtype != torch.bfloat16 or o_parts.dim() != 4 or not o_parts.is_contiguous():
+        raise TypeError("o_parts must be a contiguous bf16 [R][n_q][16][128] tensor")
+    r, n_q = o_parts.shape[0], o_parts.shape[1]
+    if lse_parts.dtype != torch.float32 or tuple(lse_parts.shape) != (r, HEADS, n_q) or \
+            not lse_parts.is_contiguous():
+        raise TypeError("lse_parts must be a contiguous fp32 [R][16][n_q] tensor")
+    if o is None:
+        o = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device)
+    _check(lib.nomas_attention_merge(o_parts.data_ptr(), lse_parts.data_ptr(), r, n_q,
+                                     o.data_ptr(), _ptr(lse), HEADS, HEAD_DIM, _stream(stream)))
+    return o
+
+
+def shard_rows(n: int, rank: int, world: int, align: int = 1):
+    """Contiguous share [a, b) of n rows for `rank` (boundaries on multiples of align)."""
+    units = (n + align - 1) // align
+    a = (units * rank) // world * align
+    b = min(n, (units * (rank + 1)) // world * align)
+    return min(a, n), b
+
+
+def sharded_segment_attention(q, local_spans, group=None, lse=None, attend=None, merge=None):
+    """Attention over keys spread across the ranks of `group` (cache sequence
+    parallelism): every rank attends with all of q over its own key spans,
+    the partial (O, LSE) of all ranks are all-gathered, and each rank merges
+    them into the full result.  `attend` and `merge` default to this
+    library's kernels (segment_attention, attention_merge)."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    n_q = q.shape[0]
+    attend = attend or (lambda qq, spans, l: segment_attention(qq, spans, lse=l))
+    merge = merge or (lambda op, lp, l: attention_merge(op, lp, lse=l))
+    part_lse = torch.empty(HEADS * n_q, dtype=torch.float32, device=q.device)
+    part_o = attend(q, local_spans, part_lse)
+    if world == 1:
+        o_parts, lse_parts = part_o[None], part_lse.view(1, HEADS, n_q)
+    else:
+        o_parts = torch.empty((world,) + tuple(part_o.shape), dtype=part_o.dtype, device=q.device)
+        lse_parts = torch.empty((world, HEADS, n_q), dtype=torch.float32, device=q.device)
+        dist.all_gather(list(o_parts.unbind(0)), part_o.contiguous(), group=group)
+        dist.all_gather(list(lse_parts.unbind(0)), part_lse.view(HEADS, n_q), group=group)
+    return merge(o_parts, lse_parts, lse)

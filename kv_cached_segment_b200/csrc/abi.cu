@@ -413,6 +413,31 @@ nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t 
                        dev_err, stream);
 }
 
+nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,
+                                   int64_t n_q, void *o, float *lse, int32_t heads,
+                                   int32_t head_dim, void *stream) {
+  nomas_status st = check_shape(heads, head_dim);
+  if (st != NOMAS_OK) return st;
+  if (n_parts <= 0 || n_q < 0 || n_q > 0x7fff0000LL)
+    return fail(NOMAS_ERR_INVALID_ARG, "need n_parts >= 1 and 0 <= n_q < 2^31");
+  if (n_q == 0) return ok();
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr || !aligned16(o_parts) ||
+      !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(NOMAS_ERR_INVALID_ARG, "merge pointers missing or misaligned");
+  const int64_t pb = (int64_t)n_parts * n_q * kRowBytes, lb = (int64_t)n_parts * n_q * kHeads * 4;
+  const int64_t ob = n_q * kRowBytes, olb = n_q * kHeads * 4;
+  if (overlap(o, ob, o_parts, pb) || overlap(o, ob, lse_parts, lb) ||
+      (lse != nullptr && (overlap(lse, olb, o_parts, pb) || overlap(lse, olb, lse_parts, lb) ||
+                          overlap(lse, olb, o, ob))))
+    return fail(NOMAS_ERR_INVALID_ARG, "merge outputs overlap the inputs");
+  const cudaError_t e = launch_merge(static_cast<const uint16_t *>(o_parts), lse_parts, n_parts,
+                                     n_q, static_cast<uint16_t *>(o), lse,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
 nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_span *spans,
                                      int32_t n_spans, void *o, float *lse, float softmax_scale,
                                      int32_t heads, int32_t head_dim, int32_t *dev_err,

@@ -96,4 +96,8 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
                                    cudaStream_t stream);
 
+// ---------------------------------------------------------------- merge ----
+cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_t n_parts,
+                         int64_t n_q, uint16_t *o, float *lse, cudaStream_t stream);
+
 }  // namespace nomas

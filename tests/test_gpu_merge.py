@@ -1,0 +1,57 @@
+"""Merging attention partials over key shards, and the sharded path on one GPU."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cached_segment_b200 as nm
+import oracle
+from seeded_inputs import randn_bf16
+from tests._util import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def test_merge_kernel_matches_oracle_formula():
+    g = torch.Generator().manual_seed(3)
+    r, n_q = 5, 300
+    o_parts = randn_bf16((r, n_q, 16, 128), 7)
+    lse_parts = torch.randn((r, 16, n_q), generator=g) * 4
+    lse_parts[2] = -float("inf")            # an empty shard
+    lse_parts[:, 3, :10] = -float("inf")    # rows where every shard is empty
+    lse = torch.empty(16 * n_q, dtype=torch.float32, device="cuda")
+    o = nm.attention_merge(o_parts.cuda(), lse_parts.cuda(), lse=lse)
+    torch.cuda.synchronize()
+    want_o, want_l = oracle.merge_partials(f64(o_parts), lse_parts.double().numpy())
+    assert_close(f64(o), want_o, max_abs=1e-2, mean_abs=1e-3, what="merged O")
+    got_l = lse.view(16, n_q).cpu().double().numpy()
+    fin = np.isfinite(want_l)
+    assert np.array_equal(np.isfinite(got_l), fin)
+    assert np.allclose(got_l[fin], want_l[fin], atol=1e-5)
+
+
+@pytest.mark.parametrize("cuts", [[0, 1000, 2500, 4000], [0, 0, 4000], [0, 1, 3999, 4000]])
+def test_sharded_keys_merge_to_full_attention(cuts):
+    q = randn_bf16((700, 16, 128), 1)
+    k = randn_bf16((4000, 16, 128), 2)
+    v = randn_bf16((4000, 16, 128), 3)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        l_r = torch.empty(16 * 700, dtype=torch.float32, device="cuda")
+        parts_o.append(nm.segment_attention(qd, [(kd[a:b], vd[a:b])], lse=l_r))
+        parts_l.append(l_r.view(16, 700))
+    lse = torch.empty(16 * 700, dtype=torch.float32, device="cuda")
+    o = nm.attention_merge(torch.stack(parts_o), torch.stack(parts_l), lse=lse)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attention(f64(q), [(f64(k), f64(v))])
+    assert_close(f64(o), o_ref, what="sharded O")
+    assert_close(lse.view(16, -1).cpu().double().numpy(), l_ref, what="sharded LSE")
+
+
+def test_sharded_attention_single_rank_is_plain_attention():
+    q = randn_bf16((300, 16, 128), 4).cuda()
+    spans = [(randn_bf16((500, 16, 128), 5).cuda(), randn_bf16((500, 16, 128), 6).cuda())]
+    o1 = nm.sharded_segment_attention(q, spans)
+    o2 = nm.segment_attention(q, spans)
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= 2 ** -7
