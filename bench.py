@@ -190,33 +190,28 @@ class LayerStep:
     def flops(self) -> float:
         return self.sparse_flops if self.sparse is not None else self.w.attention_flops()
 
-    def run(self, ev=None):
+    def run(self, ev=None, bufs=None):
         nm, w = self.nm, self.w
         ns = w.n_seg
+        q, k, v, o = (self.q, self.k, self.v, self.o) if bufs is None else bufs
         self.cache.len = w.n_cache
-        nm.kvcache_append(self.cache, self.k[:ns], self.v[:ns], q_in=self.q, q_out=self.q_rot,
+        nm.kvcache_append(self.cache, k[:ns], v[:ns], q_in=q, q_out=self.q_rot,
                           layout=self.layout, cfg=self.cfg)
         if self.frames is not None:
             nm.kvcache_select(self.cache, self.frames, self.window)
             hist = self.window.span()
         else:
             hist = self.cache.span(0, w.n_cache)
-        spans = [hist, (self.k[ns:], self.v[ns:]), self.cache.span(w.n_cache, w.n_cache + ns)]
+        spans = [hist, (k[ns:], v[ns:]), self.cache.span(w.n_cache, w.n_cache + ns)]
         if ev is not None:
             ev[0].record()
         if self.sparse is not None:
-            nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=self.o, lse=self.lse,
+            nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=o, lse=self.lse,
                                         dev_err=self.err)
         else:
-            nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
+            nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
         if ev is not None:
             ev[1].record()
-
-    def host_inputs(self):
-        """Pinned host copies of one step's inputs (for the end-to-end leg)."""
-        t = self.torch
-        return {n: getattr(self, n).cpu().pin_memory() for n in ("q", "k", "v")}, \
-            t.empty_like(self.o, device="cpu").pin_memory()
 
 
 class LayerStepI8:
@@ -263,25 +258,20 @@ class LayerStepI8:
     def flops(self) -> float:
         return self.w.attention_flops()
 
-    def run(self, ev=None):
+    def run(self, ev=None, bufs=None):
         nm, w = self.nm, self.w
         ns = w.n_seg
+        q, k, v, o = (self.q, self.k, self.v, self.o) if bufs is None else bufs
         self.cache.len = w.n_cache
-        nm.rope3d_qk(self.q, self.k, self.q_rot, self.k_rot, self.layout, self.cfg)
-        nm.kvcache_append_i8(self.cache, self.k_rot[:ns], self.v[:ns])
+        nm.rope3d_qk(q, k, self.q_rot, self.k_rot, self.layout, self.cfg)
+        nm.kvcache_append_i8(self.cache, self.k_rot[:ns], v[:ns])
         nm.kvcache_select(self.cache, self.frames, self.window)
-        spans = [self.window.span(), (self.k_rot[ns:], self.v[ns:]),
-                 (self.k_rot[:ns], self.v[:ns])]
+        spans = [self.window.span(), (self.k_rot[ns:], v[ns:]), (self.k_rot[:ns], v[:ns])]
         if ev is not None:
             ev[0].record()
-        nm.segment_attention(self.q_rot, spans, o=self.o, lse=self.lse, dev_err=self.err)
+        nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
         if ev is not None:
             ev[1].record()
-
-    def host_inputs(self):
-        t = self.torch
-        return {n: getattr(self, n).cpu().pin_memory() for n in ("q", "k", "v")}, \
-            t.empty_like(self.o, device="cpu").pin_memory()
 
 
 class SweepStep:
@@ -343,9 +333,6 @@ class SweepStep:
             nm.segment_attention(self.q_rot, spans, o=self.o, dev_err=self.err)
         if ev is not None:
             ev[1].record()
-
-    def host_inputs(self):
-        raise NotImplementedError
 
 
 def max_over_ranks(values, world: int, device):
@@ -498,26 +485,23 @@ def main():
     value = flops * args.steps * world / (ms / 1e3) / 1e12
     attn_tflops = flops / (attn_ms / 1e3) / 1e12
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs from pinned host memory and reads its output back;
+    # two buffer sets and two copy streams overlap step i+1's upload and step
+    # i-1's download with step i's kernels.
     e2e = None
     if not args.no_e2e and args.workload != "sweep":
-        host_in, host_o = step.host_inputs()
-        for _ in range(2):
-            run_e2e(step, host_in, host_o)
+        pipe = E2EPipeline(step)
+        pipe.run(2)
         torch.cuda.synchronize()
         barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, min(args.steps, 20))
-        e0.record()
-        for _ in range(n_e2e):
-            run_e2e(step, host_in, host_o)
-        e1.record()
-        torch.cuda.synchronize()
-        (e_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, "cuda")
-        h2d = sum(x.numel() * x.element_size() for x in host_in.values())
+        e_ms = pipe.run(n_e2e)
+        (e_ms,) = max_over_ranks([e_ms], world, "cuda")
         e2e = {"value": flops * n_e2e * world / (e_ms / 1e3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": host_o.numel() * 2,
-               "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
+               "h2d_bytes_per_step": pipe.h2d_bytes, "d2h_bytes_per_step": pipe.d2h_bytes,
+               "ms_per_step": e_ms / n_e2e, "steps": n_e2e,
+               "overlap": "double-buffered inputs/outputs, separate H2D and D2H streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "sweep":
@@ -568,12 +552,66 @@ def main():
     print(json.dumps(out), flush=True)
 
 
-def run_e2e(step, host_in, host_o):
-    step.q.copy_(host_in["q"], non_blocking=True)
-    step.k.copy_(host_in["k"], non_blocking=True)
-    step.v.copy_(host_in["v"], non_blocking=True)
-    step.run()
-    host_o.copy_(step.o, non_blocking=True)
+class E2EPipeline:
+    """End-to-end steps through the public API from pinned host buffers."""
+
+    def __init__(self, step):
+        import torch
+
+        self.torch, self.step = torch, step
+        self.host_in = [{n: getattr(step, n).cpu().pin_memory() for n in ("q", "k", "v")}
+                        for _ in range(2)]
+        self.host_o = [torch.empty_like(step.o, device="cpu").pin_memory() for _ in range(2)]
+        self.dev = [(step.q, step.k, step.v, step.o),
+                    (torch.empty_like(step.q), torch.empty_like(step.k),
+                     torch.empty_like(step.v), torch.empty_like(step.o))]
+        self.h2d_bytes = sum(x.numel() * x.element_size() for x in self.host_in[0].values())
+        self.d2h_bytes = step.o.numel() * step.o.element_size()
+        self.s_h2d = torch.cuda.Stream()
+        self.s_d2h = torch.cuda.Stream()
+
+    def run(self, n: int) -> float:
+        """Runs n steps; returns elapsed ms from the first upload to the last download."""
+        torch = self.torch
+        comp = torch.cuda.current_stream()
+        ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+        in_ready = [ev(), ev()]
+        done = [ev(), ev()]
+        out_read = [ev(), ev()]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(comp)
+        self.s_h2d.wait_event(start)
+        self.s_d2h.wait_event(start)
+
+        def upload(i):
+            b = i % 2
+            with torch.cuda.stream(self.s_h2d):
+                if i >= 2:
+                    self.s_h2d.wait_event(done[b])  # step i-2 no longer reads buffer b
+                q, k, v, _ = self.dev[b]
+                q.copy_(self.host_in[b]["q"], non_blocking=True)
+                k.copy_(self.host_in[b]["k"], non_blocking=True)
+                v.copy_(self.host_in[b]["v"], non_blocking=True)
+                in_ready[b].record(self.s_h2d)
+
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            comp.wait_event(in_ready[b])
+            if i >= 2:
+                comp.wait_event(out_read[b])  # step i-2's output has been read back
+            self.step.run(bufs=self.dev[b])
+            done[b].record(comp)
+            with torch.cuda.stream(self.s_d2h):
+                self.s_d2h.wait_event(done[b])
+                self.host_o[b].copy_(self.dev[b][3], non_blocking=True)
+                out_read[b].record(self.s_d2h)
+        stop.record(self.s_d2h)
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop)
 
 
 def run_reference(args, rank, world):
