@@ -583,83 +583,104 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           break;
         }
         tc_fence_after();
-        // S row in two halves: the max of the first half overlaps the load
-        // of the second.
+        // The whole S row (128 keys) comes out of TMEM in one go.
         uint32_t sr[128];
         tmem::ld32(tS + 0, sr + 0);
         tmem::ld32(tS + 32, sr + 32);
-        tmem::wait_ld64(sr);
         tmem::ld32(tS + 64, sr + 64);
         tmem::ld32(tS + 96, sr + 96);
+        tmem::wait_ld128(sr);
         float *sv = reinterpret_cast<float *>(sr);
         const int64_t rem = len - (int64_t)kt * kBN;
         const int valid = rem < kBN ? (int)rem : kBN;
         if (valid < kBN) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 128; ++c)
             if (c >= valid) sv[c] = -INFINITY;
         }
-        float mA = -INFINITY, mB = -INFINITY, mC = -INFINITY, mD = -INFINITY;
+        auto row_max = [&](int c0, int c1) {
+          float mA = -INFINITY, mB = -INFINITY, mC = -INFINITY, mD = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          mA = fmax3(mA, sv[c], sv[c + 1]);
-          mB = fmax3(mB, sv[c + 2], sv[c + 3]);
-          mC = fmax3(mC, sv[c + 4], sv[c + 5]);
-          mD = fmax3(mD, sv[c + 6], sv[c + 7]);
-        }
-        tmem::wait_ld64(sr + 64);
-        if (valid < kBN) {
-#pragma unroll
-          for (int c = 64; c < 128; ++c)
-            if (c >= valid) sv[c] = -INFINITY;
-        }
-#pragma unroll
-        for (int c = 64; c < 128; c += 8) {
-          mA = fmax3(mA, sv[c], sv[c + 1]);
-          mB = fmax3(mB, sv[c + 2], sv[c + 3]);
-          mC = fmax3(mC, sv[c + 4], sv[c + 5]);
-          mD = fmax3(mD, sv[c + 6], sv[c + 7]);
-        }
-        const float mx = fmaxf(fmax3(mA, mB, mC), mD) * sl2;
-        // Lazy max: raise it (and rescale O and l by alpha) only when some
-        // row of the warp grew by more than 2^8; the O update happens once
-        // the first half of P is stored, when its S values are no longer live.
+          for (int c = c0; c < c1; c += 8) {
+            mA = fmax3(mA, sv[c], sv[c + 1]);
+            mB = fmax3(mB, sv[c + 2], sv[c + 3]);
+            mC = fmax3(mC, sv[c + 4], sv[c + 5]);
+            mD = fmax3(mD, sv[c + 6], sv[c + 7]);
+          }
+          return fmaxf(fmax3(mA, mB, mC), mD) * sl2;
+        };
         bool rescale = false;
         float alpha = 1.f;
-        if (j == 0) {
-          m = mx;
-        } else if (__any_sync(0xffffffffu, mx > m + 8.0f)) {
-          const float m_new = fmaxf(m, mx);
-          alpha = ex2(m - m_new);
-          m = m_new;
-          l *= alpha;
-          rescale = true;
-        }
+        if (j == 0) m = row_max(0, 128);
         // P = 2^(s * scale * log2 e - m) as bf16 pairs, published to the MMA
         // lane in two halves of 64 keys so that O += P V on the first half
         // overlaps the exponentials of the second.  The row sum accumulates
-        // the fp32 values.  A pending O rescale happens before the first
-        // half is published (the MMA lane may then start updating O).
-        const uint64_t sl2x2 = f2(sl2, sl2), negm2 = f2(-m, -m);
-        uint64_t lacc0 = f2(0.f, 0.f), lacc1 = f2(0.f, 0.f);
+        // the fp32 values.
+        uint64_t lacc0, lacc1;
         uint32_t pk0[32], pk1[32];
+        float xp;  // max exponent fed to the FMA-pipe exp2 in half 0
+        auto half0 = [&]() {
+          const uint64_t sl2x2 = f2(sl2, sl2), negm2 = f2(-m, -m);
+          lacc0 = f2(0.f, 0.f);
+          lacc1 = f2(0.f, 0.f);
+          xp = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const uint64_t x = fma2(f2(sv[2 * c], sv[2 * c + 1]), sl2x2, negm2);
-          uint64_t e;
-          if (pair_on_fma(c)) {
-            e = exp2_poly_x2(x);
-          } else {
-            const float2 xv = unf2(x);
-            e = f2(ex2(xv.x), ex2(xv.y));
+          for (int c = 0; c < 32; ++c) {
+            const uint64_t x = fma2(f2(sv[2 * c], sv[2 * c + 1]), sl2x2, negm2);
+            uint64_t e;
+            if (pair_on_fma(c)) {
+              const float2 xv = unf2(x);
+              xp = fmax3(xp, xv.x, xv.y);
+              e = exp2_poly_x2(x);
+            } else {
+              const float2 xv = unf2(x);
+              e = f2(ex2(xv.x), ex2(xv.y));
+            }
+            if (c & 1)
+              lacc1 = add2(lacc1, e);
+            else
+              lacc0 = add2(lacc0, e);
+            const float2 ev = unf2(e);
+            pk0[c] = pack_bf16x2(ev.x, ev.y);
           }
-          if (c & 1)
-            lacc1 = add2(lacc1, e);
-          else
-            lacc0 = add2(lacc0, e);
-          const float2 ev = unf2(e);
-          pk0[c] = pack_bf16x2(ev.x, ev.y);
+        };
+        // Stale max: after the first tile, half 0 is exponentiated against
+        // the running max m without first taking this tile's max.  The
+        // result is exact for any m (the factor 2^-m cancels in O / l); m
+        // only has to keep every P far from overflow.  Three bounds, each
+        // P <= 2^16, are checked afterwards:
+        //   - the fp32 sum of half 0 (the hardware exp2 returns +inf on
+        //     overflow, which fails the test too);
+        //   - the max of the half-0 columns whose exp2 runs on the FMA pipe,
+        //     since that emulation is only valid for arguments below 128;
+        //   - the max of half 1, before it is exponentiated.
+        // If any row of the warp fails, the exact max is taken, O and l are
+        // rescaled and half 0 is redone; S is still intact in TMEM then.
+        half0();
+        if (j > 0) {
+          const float mx1 = row_max(64, 128);
+          const float2 a0 = unf2(lacc0), a1 = unf2(lacc1);
+          const float lh0 = (a0.x + a0.y) + (a1.x + a1.y);
+          const bool bad = !(lh0 <= 65536.f) || xp > 16.f || mx1 > m + 16.f;
+          if (__any_sync(0xffffffffu, bad)) {
+            tmem::ld32(tS + 0, sr + 0);
+            tmem::ld32(tS + 32, sr + 32);
+            tmem::wait_ld64(sr);
+            if (valid < 64) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c)
+                if (c >= valid) sv[c] = -INFINITY;
+            }
+            const float m_new = fmaxf(m, row_max(0, 128));
+            alpha = ex2(m - m_new);
+            m = m_new;
+            l *= alpha;
+            rescale = true;
+            half0();
+          }
         }
+        // A pending O rescale happens before the first half is published
+        // (the MMA lane may then start updating O).
         tmem::st32(tS + 0, pk0);
         if (rescale) {
 #pragma unroll
@@ -675,6 +696,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
         }
         tmem::wait_st();
         tc_fence_before();
+        const uint64_t sl2x2 = f2(sl2, sl2), negm2 = f2(-m, -m);
         mbar_arrive(bar(kBarPHalf + tile));
 #pragma unroll
         for (int c = 32; c < 64; ++c) {

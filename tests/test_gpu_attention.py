@@ -208,3 +208,19 @@ def test_wait_timeout_is_reported_and_context_survives():
     assert torch.all(o == 7.0)  # aborted blocks write no output
     # the same context still computes correct results
     _check(q, spans, what="after timeout")
+
+
+@pytest.mark.parametrize("col", [2, 5, 17, 66])
+@pytest.mark.parametrize("spike", [100.0, 300.0])
+def test_attention_logit_spike_in_later_tile(col, spike):
+    # One key, in the second 128-key tile, scores `spike` (natural-log units)
+    # above the others, so the softmax is that key's V row.  Its column lands
+    # on exponentials computed on either pipe and in either half of the tile:
+    # a running max that is not raised in time would overflow there.
+    n_k = 400
+    q = torch.ones((64, 16, 128), dtype=torch.bfloat16)
+    k = randn_bf16((n_k, 16, 128), 50)
+    k[128 + col] = spike / math.sqrt(128.0)
+    v = randn_bf16((n_k, 16, 128), 51)
+    o = _check(q, [(k, v)], what=f"spike {spike} at column {col}")
+    assert_close(f64(o), np.broadcast_to(f64(v[128 + col]), (64, 16, 128)), what="spike row")
