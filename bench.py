@@ -65,7 +65,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("attention.cu", "tmem_ops.cuh", "nomas_internal.h"):
+    for name in ("attention.cu", "f32x2.cuh", "tmem_ops.cuh", "nomas_internal.h"):
         with open(os.path.join(ROOT, "kv_cached_segment_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

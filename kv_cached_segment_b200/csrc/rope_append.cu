@@ -47,41 +47,72 @@ __device__ __forceinline__ uint4 rot_chunk(uint4 v, const float (&c)[4], const f
   return v;
 }
 
-// Symmetric INT8 quantisation of one (token, head): the 16 threads of the row
-// each hold 8 of the 128 bf16 values; the absmax a is reduced with shuffles
-// inside the row's 16 lanes.  The stored scale is a / 127 and code =
-// rint(x * (127 / a)); the two divisions (one per token and head) and the
-// product round to nearest in float32 and the conversion rounds half to even,
-// so the codes are reproducible bit for bit; an all-zero head gets scale 0.
-__device__ __forceinline__ uint2 quant_chunk(uint4 v, unsigned row_mask, float *scale_out) {
+// Symmetric INT8 quantisation per (token, head): stored scale = a / 127 and
+// code = rint(x * (127 / a)) with a = max |x| over the head's 128 values; the
+// two divisions and the product round to nearest in float32 and rint rounds
+// half to even, so the codes are reproducible bit for bit; an all-zero head
+// gets scale 0 and codes 0.
+//
+// A thread holds 8 values of each of 4 items (the keys, or the values, of 4
+// heads) of its row.  The absmax of the 4 items over the row's 16 lanes is a
+// transposed butterfly: at the first two xor steps a lane keeps half of its
+// items and trades the other half with its partner, so 2 + 1 + 1 + 1
+// shuffles leave lanes 4i..4i+3 holding item i reduced over the row.  Each
+// lane then does the divisions for its own item only, and 4 shuffles hand
+// every lane the reciprocal of each item.
+static_assert(kHeadGroup == 4, "the butterfly below reduces 4 items over 16 lanes");
+
+__device__ __forceinline__ float chunk_absmax(uint4 v) {
+  const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xffff0000u);
+  const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xffff0000u);
+  const float x4 = __uint_as_float(v.z << 16), x5 = __uint_as_float(v.z & 0xffff0000u);
+  const float x6 = __uint_as_float(v.w << 16), x7 = __uint_as_float(v.w & 0xffff0000u);
+  float m = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fabsf(x2));
+  m = fmaxf(fmaxf(m, fabsf(x3)), fabsf(x4));
+  m = fmaxf(fmaxf(m, fabsf(x5)), fabsf(x6));
+  return fmaxf(m, fabsf(x7));
+}
+
+// Item (cc >> 2)'s absmax over the 16 lanes of the row.
+__device__ __forceinline__ float row_absmax_transposed(const float (&am)[kHeadGroup], int cc,
+                                                       unsigned row_mask) {
+  const bool b8 = cc & 8, b4 = cc & 4;
+  float a1[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float keep = b8 ? am[j + 2] : am[j];
+    const float send = b8 ? am[j] : am[j + 2];
+    a1[j] = fmaxf(keep, __shfl_xor_sync(row_mask, send, 8));
+  }
+  const float keep = b4 ? a1[1] : a1[0];
+  const float send = b4 ? a1[0] : a1[1];
+  float r = fmaxf(keep, __shfl_xor_sync(row_mask, send, 4));
+  r = fmaxf(r, __shfl_xor_sync(row_mask, r, 2));
+  return fmaxf(r, __shfl_xor_sync(row_mask, r, 1));
+}
+
+// 8 codes of one chunk.  |x * inv| <= 127 (1 + 2^-24)^2 < 127.5, so adding
+// 1.5 * 2^23 rounds the product to an integer half to even and leaves it,
+// in two's complement, in the low byte of the sum; no clamp is needed.  The
+// product must be rounded to float32 before the add (a fused multiply-add
+// would round x * (127 / a) = 63.5 - tiny, common when x = a / 2, down to
+// 63 instead of 63.5 -> 64; a version written with the packed f32x2
+// multiply and add gave exactly those codes), so both steps use the scalar
+// intrinsics that are never contracted.
+__device__ __forceinline__ uint2 quant_chunk(uint4 v, float inv) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float x[8];
+  uint32_t t[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    t[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w[i] << 16), inv), kMagic));
+    t[2 * i + 1] =
+        __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w[i] & 0xffff0000u), inv), kMagic));
   }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(row_mask, amax, off));
-  const float scale = __fdiv_rn(amax, 127.f);
-  uint32_t lo = 0, hi = 0;
-  if (amax > 0.f) {
-    const float inv = __fdiv_rn(127.f, amax);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int q = __float2int_rn(__fmul_rn(x[i], inv));
-      q = max(-127, min(127, q));
-      const uint32_t b = (uint32_t)(q & 0xff);
-      if (i < 4)
-        lo |= b << (8 * i);
-      else
-        hi |= b << (8 * (i - 4));
-    }
-  }
-  *scale_out = scale;
+  const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040),
+                                  0x5410);
   return make_uint2(lo, hi);
 }
 
@@ -125,39 +156,73 @@ rope_append_kernel(const __grid_constant__ RopeArgs a) {
   uint4 *k_out = reinterpret_cast<uint4 *>(a.k_out);
   uint4 *v_out = reinterpret_cast<uint4 *>(a.v_out);
 
+  if constexpr (!kQuant) {
 #pragma unroll 1
-  for (int h0 = 0; h0 < kHeads; h0 += kHeadGroup) {
-    uint4 qv[kHeadGroup], kv[kHeadGroup], vv[kHeadGroup];
+    for (int h0 = 0; h0 < kHeads; h0 += kHeadGroup) {
+      uint4 qv[kHeadGroup], kv[kHeadGroup], vv[kHeadGroup];
 #pragma unroll
-    for (int g = 0; g < kHeadGroup; ++g) {
-      const int64_t off = base + (int64_t)(h0 + g) * 16;
-      if (do_q) qv[g] = q_in[off];
-      if (do_k) kv[g] = k_in[off];
-      if (do_v) vv[g] = v_in[off];
-    }
+      for (int g = 0; g < kHeadGroup; ++g) {
+        const int64_t off = base + (int64_t)(h0 + g) * 16;
+        if (do_q) qv[g] = q_in[off];
+        if (do_k) kv[g] = k_in[off];
+        if (do_v) vv[g] = v_in[off];
+      }
 #pragma unroll
-    for (int g = 0; g < kHeadGroup; ++g) {
-      const int64_t off = base + (int64_t)(h0 + g) * 16;
-      if (do_q) q_out[off] = rotate ? rot_chunk(qv[g], c, s) : qv[g];
-      if constexpr (kQuant) {
-        // codes: 8 bytes per thread at [row][head][8cc..8cc+7]; one scale per (row, head)
-        const int64_t coff = row * (kRowElems / 8) + (int64_t)(h0 + g) * 16 + cc;
-        const int64_t soff = row * kHeads + h0 + g;
-        float sc;
-        if (do_k) {
-          const uint2 q8 = quant_chunk(rotate ? rot_chunk(kv[g], c, s) : kv[g], row_mask, &sc);
-          reinterpret_cast<uint2 *>(a.k_codes)[coff] = q8;
-          if (cc == 0) a.k_scales[soff] = sc;
-        }
-        if (do_v) {
-          const uint2 q8 = quant_chunk(vv[g], row_mask, &sc);
-          reinterpret_cast<uint2 *>(a.v_codes)[coff] = q8;
-          if (cc == 0) a.v_scales[soff] = sc;
-        }
-      } else {
+      for (int g = 0; g < kHeadGroup; ++g) {
+        const int64_t off = base + (int64_t)(h0 + g) * 16;
+        if (do_q) q_out[off] = rotate ? rot_chunk(qv[g], c, s) : qv[g];
         if (do_k) k_out[off] = rotate ? rot_chunk(kv[g], c, s) : kv[g];
         if (do_v) v_out[off] = vv[g];
       }
+    }
+  } else {
+    // Q rows first (rotated, bf16), then K and V into the INT8 cache, so
+    // that the quantiser's loop holds no Q registers.
+    if (do_q) {
+#pragma unroll 1
+      for (int h0 = 0; h0 < kHeads; h0 += kHeadGroup) {
+        uint4 qv[kHeadGroup];
+#pragma unroll
+        for (int g = 0; g < kHeadGroup; ++g) qv[g] = q_in[base + (int64_t)(h0 + g) * 16];
+#pragma unroll
+        for (int g = 0; g < kHeadGroup; ++g)
+          q_out[base + (int64_t)(h0 + g) * 16] = rotate ? rot_chunk(qv[g], c, s) : qv[g];
+      }
+    }
+    if (!do_k && !do_v) return;  // uniform over the row's 16 lanes
+#pragma unroll 1
+    for (int h0 = 0; h0 < kHeads; h0 += kHeadGroup) {
+      uint4 kv[kHeadGroup], vv[kHeadGroup];
+#pragma unroll
+      for (int g = 0; g < kHeadGroup; ++g) {
+        const int64_t off = base + (int64_t)(h0 + g) * 16;
+        if (do_k) kv[g] = k_in[off];
+        if (do_v) vv[g] = v_in[off];
+      }
+      // Keys (rotated and rounded to bf16 first), then values: per pass the
+      // 4 heads of the group are the butterfly's 4 items.
+      auto quant_pass = [&](const uint4 (&src)[kHeadGroup], int8_t *codes, float *scales) {
+        float am[kHeadGroup];
+#pragma unroll
+        for (int g = 0; g < kHeadGroup; ++g) am[g] = chunk_absmax(src[g]);
+        const float amax = row_absmax_transposed(am, cc, row_mask);
+        const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+        if ((cc & 3) == 0) scales[row * kHeads + h0 + (cc >> 2)] = __fdiv_rn(amax, 127.f);
+#pragma unroll
+        for (int g = 0; g < kHeadGroup; ++g) {
+          // 8 codes per thread at [row][head][8cc..8cc+7]
+          const int64_t coff = row * (kRowElems / 8) + (int64_t)(h0 + g) * 16 + cc;
+          const float inv_g = __shfl_sync(row_mask, inv, (threadIdx.x & 16) + 4 * g);
+          reinterpret_cast<uint2 *>(codes)[coff] = quant_chunk(src[g], inv_g);
+        }
+      };
+      if (do_k) {
+#pragma unroll
+        for (int g = 0; g < kHeadGroup; ++g)
+          if (rotate) kv[g] = rot_chunk(kv[g], c, s);
+        quant_pass(kv, a.k_codes, a.k_scales);
+      }
+      if (do_v) quant_pass(vv, a.v_codes, a.v_scales);
     }
   }
 }

@@ -55,6 +55,8 @@ def test_append_rotated_keys_within_quantisation_error():
     assert np.array_equal(_codes(cache.v), want_c)
     assert np.array_equal(cache.v_scale.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
     assert_close(f64(q_out[:ns]), oracle.rope3d(f64(q), ns, t, h, w)[:ns], what="Q'")
+    # text rows of Q are not rotated: copied bit for bit
+    assert np.array_equal(bits(q_out[ns:]), bits(q[ns:]))
 
 
 def _i8_source(n_frames, tpf, seed):
