@@ -535,8 +535,9 @@ def main():
                   f"{attn_per_step * (w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
             "parallelism": f"independent layer-step per GPU x{world}",
         },
-        "pct_of_measured_bf16_peak": 100.0 * value / peak,
-        "pct_of_datasheet_bf16_peak": 100.0 * value / DATASHEET_BF16_TFLOPS,
+        # per GPU: value is the whole job's aggregate over `world` GPUs
+        "pct_of_measured_bf16_peak": 100.0 * value / world / peak,
+        "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
         "attention_ms": attn_ms / attn_per_step,
         "roofline": {"kernel": "attention_kernel", "bound": "tensor",
                      "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
