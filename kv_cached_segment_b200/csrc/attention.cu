@@ -275,7 +275,7 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
 
 // Pairs of P (out of every 8) whose exponentials run on the FMA pipe.
 #ifndef NOMAS_EXP2_FMA_PAIRS
-#define NOMAS_EXP2_FMA_PAIRS 2
+#define NOMAS_EXP2_FMA_PAIRS 1
 #endif
 #ifndef NOMAS_EXP2_FMA_PAIRS_H1
 #define NOMAS_EXP2_FMA_PAIRS_H1 NOMAS_EXP2_FMA_PAIRS

@@ -210,7 +210,7 @@ def test_wait_timeout_is_reported_and_context_survives():
     _check(q, spans, what="after timeout")
 
 
-@pytest.mark.parametrize("col", [2, 5, 17, 66])
+@pytest.mark.parametrize("col", [2, 5, 17, 64, 66])
 @pytest.mark.parametrize("spike", [100.0, 300.0])
 def test_attention_logit_spike_in_later_tile(col, spike):
     # One key, in the second 128-key tile, scores `spike` (natural-log units)
