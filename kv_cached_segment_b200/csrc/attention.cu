@@ -27,13 +27,15 @@
 //   O0 += P0(j) V_j ; S0 = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1 = Q1 K_{j+1}^T
 // so each softmax group works on one tile while the tensor core runs the
 // other tile's two GEMMs.  P is published in two halves of 64 keys, so the
-// first half of O += P V runs while the softmax computes the second half.  tcgen05 operations of one thread complete in issue
-// order, so the commit that announces S_i(j+1) also covers O_i += P_i(j) V_j:
-// when a softmax thread sees S_i ready, O_i is quiescent and the thread may
-// rescale it in place.  Rescaling is lazy: the running max is only raised
-// when a row's new max exceeds it by more than 2^8 (log2 domain), otherwise P
-// is formed against the stale max (values up to 256) and the final division
-// by the row sum, formed with the same max, makes the result exact.
+// first half of O += P V runs while the softmax computes the second half.
+// tcgen05 operations of one thread complete in issue order, so the commit
+// that announces S_i(j+1) also covers O_i += P_i(j) V_j: when a softmax
+// thread sees S_i ready, O_i is quiescent and the thread may rescale it in
+// place.  The running max is allowed to be stale: P is formed against it
+// (values up to 2^16) and the final division by the row sum, formed with the
+// same max, makes the result exact; it is raised, with O and the row sum
+// rescaled, only when a bound check shows that some P of the tile would
+// exceed 2^16.
 //
 // Every wait is bounded (a globaltimer limit); on expiry the kernel records
 // NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and
