@@ -49,6 +49,10 @@ def parse_args():
     p.add_argument("--sparse", type=float, default=0.0,
                    help="block-sparse attention keeping this fraction of the video key tiles "
                         "(text tiles always kept); 0 = dense")
+    p.add_argument("--key-shards", type=int, default=0,
+                   help="split the key sequence into this many contiguous shards, attend over "
+                        "each into a partial (O, LSE) and merge them (the per-GPU work of "
+                        "key-sharded attention, on one GPU); 0 = one launch over all keys")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -170,6 +174,34 @@ class LayerStep:
             self.frames = None
         self.launches_per_step = 3 if self.frames else 2
         self.sparse = None
+        self.shards = 0
+
+    def use_key_shards(self, n_shards: int):
+        """Attention over `n_shards` contiguous ranges of the key sequence
+        (boundaries on 128-key tiles), each into its own partial (O, LSE),
+        then one merge: what each GPU of key-sharded attention computes."""
+        torch, w = self.torch, self.w
+        self.shards = n_shards
+        self.part_o = torch.empty((n_shards, w.n_q, 16, 128), dtype=torch.bfloat16,
+                                  device="cuda")
+        self.part_lse = torch.empty((n_shards, 16, w.n_q), dtype=torch.float32, device="cuda")
+        self.merge_ev = []
+        self.launches_per_step += n_shards  # n_shards attention launches + 1 merge, was 1
+
+    def _shard_spans(self, spans):
+        lens = [int(k.shape[0]) for k, _ in spans]
+        n_k = sum(lens)
+        out = []
+        for r in range(self.shards):
+            a, b = self.nm.shard_rows(n_k, r, self.shards, align=128)
+            sub, base = [], 0
+            for (k, v), n in zip(spans, lens):
+                lo, hi = max(a, base), min(b, base + n)
+                if hi > lo:
+                    sub.append((k[lo - base:hi - base], v[lo - base:hi - base]))
+                base += n
+            out.append(sub if sub else [(spans[0][0][:0], spans[0][1][:0])])
+        return out
 
     def use_sparse(self, fraction: float, seed: int):
         """Seeded block-sparse selection: text tiles kept, `fraction` of the
@@ -213,6 +245,18 @@ class LayerStep:
         if self.sparse is not None:
             nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=o, lse=self.lse,
                                         dev_err=self.err)
+        elif self.shards:
+            for r, sub in enumerate(self._shard_spans(spans)):
+                nm.segment_attention(self.q_rot, sub, o=self.part_o[r],
+                                     lse=self.part_lse[r].view(-1), dev_err=self.err)
+            if ev is not None:
+                mev = (self.torch.cuda.Event(enable_timing=True),
+                       self.torch.cuda.Event(enable_timing=True))
+                mev[0].record()
+            nm.attention_merge(self.part_o, self.part_lse, o=o, lse=self.lse)
+            if ev is not None:
+                mev[1].record()
+                self.merge_ev.append(mev)
         else:
             nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
         if ev is not None:
@@ -407,6 +451,10 @@ def make_step(args, rank):
     step = LayerStep(args.workload, seed=1 + rank)
     if args.sparse > 0:
         step.use_sparse(args.sparse, seed=1 + rank)
+    if args.key_shards > 0:
+        if args.sparse > 0:
+            raise SystemExit("--key-shards and --sparse are exclusive")
+        step.use_key_shards(args.key_shards)
     return step
 
 
@@ -418,6 +466,9 @@ def workload_text(args, step) -> str:
                 f"{w.n_cache} cached tokens per layer)")
     hist = w.n_window if w.select_frames else w.n_cache
     extra = " (INT8 history cache)" if args.int8 else ""
+    if getattr(args, "key_shards", 0) > 0:
+        extra += (f" (keys split into {args.key_shards} contiguous shards, partial results "
+                  f"merged)")
     if args.sparse > 0:
         extra += (f" (block-sparse: text kept, {100 * args.sparse:.0f}% of video key tiles "
                   f"per 256-query block and head)")
@@ -482,9 +533,14 @@ def main():
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error word {int(step.err.item())}")
 
-    ms, attn_ms = max_over_ranks(
-        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for a, b in evs)],
+    merge_ms = 0.0
+    n_shards = getattr(step, "shards", 0)
+    if n_shards:
+        merge_ms = statistics.mean(a.elapsed_time(b) for a, b in step.merge_ev[:args.steps])
+    ms, attn_ms, merge_ms = max_over_ranks(
+        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for a, b in evs), merge_ms],
         world, "cuda")
+    attn_ms -= merge_ms  # attention launches only
     ms_per_step = ms / args.steps
     flops = step.flops()
     value = flops * args.steps * world / (ms / 1e3) / 1e12
@@ -552,6 +608,15 @@ def main():
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if n_shards:
+        # merge: R partial O rows (+ LSE) read, one O row (+ LSE) written per query row
+        mbytes = (n_shards + 1) * w.n_q * (16 * 128 * 2 + 16 * 4)
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        out["config"]["key_shards"] = n_shards
+        out["merge"] = {"kernel": "merge_kernel", "bound": "hbm", "ms": merge_ms,
+                        "bytes": mbytes, "achieved": mbytes / (merge_ms / 1e3) / 1e9,
+                        "peak": hbm, "unit": "GB/s",
+                        "frac": mbytes / (merge_ms / 1e3) / 1e9 / hbm}
     if args.workload == "sweep":
         out["ms_per_segment"] = ms_per_step * step.steps_per_segment
         out["roofline"]["note"] = "per-step average over the 54 layers (rope3d_qk launches included)"

@@ -55,6 +55,7 @@ typedef enum {
 #define NOMAS_HEADS 16
 #define NOMAS_HEAD_DIM 128
 #define NOMAS_MAX_SPANS 4
+#define NOMAS_MAX_MERGE_PARTS 32 /* partial results one attention merge combines */
 
 /*
  * 3D rotary configuration: the head dimension is split into a temporal chunk
@@ -307,6 +308,7 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
  *   o        : [n_q][heads][head_dim] bf16 output; lse: optional [heads][n_q].
  * Parts with LSE = -inf are empty and contribute nothing; if all are empty the
  * row gets O = 0 and LSE = -inf.  Outputs must not overlap the inputs.
+ * 1 <= n_parts <= NOMAS_MAX_MERGE_PARTS (more returns NOMAS_ERR_UNSUPPORTED).
  * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
  */
 nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,

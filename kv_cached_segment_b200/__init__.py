@@ -31,6 +31,7 @@ NOMAS_ERR_CUDA = 5
 DEVERR_BAD_FRAME_INDEX = 0x1
 DEVERR_WAIT_TIMEOUT = 0x2
 MAX_SPANS = 4
+MAX_MERGE_PARTS = 32
 
 EXPORTED_SYMBOLS = (
     "nomas_last_error",

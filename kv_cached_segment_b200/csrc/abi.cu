@@ -420,6 +420,8 @@ nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, 
   if (st != NOMAS_OK) return st;
   if (n_parts <= 0 || n_q < 0 || n_q > 0x7fff0000LL)
     return fail(NOMAS_ERR_INVALID_ARG, "need n_parts >= 1 and 0 <= n_q < 2^31");
+  if (n_parts > NOMAS_MAX_MERGE_PARTS)
+    return fail(NOMAS_ERR_UNSUPPORTED, "n_parts %d exceeds %d", n_parts, NOMAS_MAX_MERGE_PARTS);
   if (n_q == 0) return ok();
   if (o_parts == nullptr || lse_parts == nullptr || o == nullptr || !aligned16(o_parts) ||
       !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||

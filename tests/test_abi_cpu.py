@@ -226,3 +226,35 @@ def test_int8_append_and_select_validation(lib):
     ok_idx = (ctypes.c_int32 * 2)(0, 1)
     st = lib.nomas_kvcache_select_i8(ctypes.byref(src), ok_idx, 2, 0, ctypes.byref(overl), None, None)
     assert st == nm.NOMAS_ERR_INVALID_ARG
+
+
+def test_sparse_attention_validation(lib):
+    spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, 300))
+    o, lists, counts, err = FAKE + 3 * 10 ** 9, FAKE + 4 * 10 ** 9, FAKE + 5 * 10 ** 9, FAKE + 6 * 10 ** 9
+    f = lib.nomas_segment_attention_sparse
+    assert f(FAKE, 100, spans, 1, None, counts, 3, o, None, 0.0, 16, 128, err, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # no tile list
+    assert f(FAKE, 100, spans, 1, lists, counts, -1, o, None, 0.0, 16, 128, err, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # max_tiles < 0
+    assert f(FAKE, 100, spans, 1, lists, counts, 3, o, None, 0.0, 16, 128, None, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # a device list needs dev_err
+    assert f(FAKE, 100, spans, 1, lists + 2, counts, 3, o, None, 0.0, 16, 128, err, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # misaligned list
+    assert f(FAKE, 100, spans, 1, lists, counts, 3, o, None, 0.0, 8, 128, err, None) \
+        == nm.NOMAS_ERR_UNSUPPORTED
+
+
+def test_merge_validation(lib):
+    parts, lse_parts, o, lse = FAKE, FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, FAKE + 3 * 10 ** 9
+    f = lib.nomas_attention_merge
+    assert f(parts, lse_parts, 0, 100, o, lse, 16, 128, None) == nm.NOMAS_ERR_INVALID_ARG
+    assert f(parts, lse_parts, nm.MAX_MERGE_PARTS + 1, 100, o, lse, 16, 128, None) \
+        == nm.NOMAS_ERR_UNSUPPORTED
+    assert f(parts, lse_parts, 4, 100, o, lse, 16, 64, None) == nm.NOMAS_ERR_UNSUPPORTED
+    assert f(parts, lse_parts, 4, 100, o + 8, lse, 16, 128, None) == nm.NOMAS_ERR_INVALID_ARG
+    assert f(parts, lse_parts, 4, 100, o, lse + 2, 16, 128, None) == nm.NOMAS_ERR_INVALID_ARG
+    assert f(parts, lse_parts, 4, 100, parts + ROW, lse, 16, 128, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # output inside the partials
+    assert f(parts, lse_parts, 4, 100, o, lse_parts, 16, 128, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # merged LSE over the partial LSEs
+    assert f(parts, lse_parts, 4, 0, None, None, 16, 128, None) == nm.NOMAS_OK  # nothing to do

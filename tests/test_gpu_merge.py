@@ -11,12 +11,12 @@ from tests._util import assert_bf16_rounding, assert_close, f64
 pytestmark = pytest.mark.gpu
 
 
-def test_merge_kernel_matches_oracle_formula():
+@pytest.mark.parametrize("r,n_q", [(5, 300), (1, 17), (7, 1000), (nm.MAX_MERGE_PARTS, 129)])
+def test_merge_kernel_matches_oracle_formula(r, n_q):
     g = torch.Generator().manual_seed(3)
-    r, n_q = 5, 300
     o_parts = randn_bf16((r, n_q, 16, 128), 7)
     lse_parts = torch.randn((r, 16, n_q), generator=g) * 4
-    lse_parts[2] = -float("inf")            # an empty shard
+    lse_parts[r // 2] = -float("inf")       # an empty shard (the only one when r = 1)
     lse_parts[:, 3, :10] = -float("inf")    # rows where every shard is empty
     lse = torch.empty(16 * n_q, dtype=torch.float32, device="cuda")
     o = nm.attention_merge(o_parts.cuda(), lse_parts.cuda(), lse=lse)
