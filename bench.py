@@ -41,7 +41,8 @@ def parse_args():
     p.add_argument("--steps", type=int, default=40)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["nomas", "reference"], default="nomas")
-    p.add_argument("--workload", choices=["720p", "bounded", "short", "mid", "tiny", "sweep"],
+    p.add_argument("--workload", choices=["720p", "bounded", "bounded90", "short", "mid", "tiny",
+                                          "sweep"],
                    default="720p")
     p.add_argument("--int8", action="store_true",
                    help="bounded workload with an INT8 history cache (quantising append, "

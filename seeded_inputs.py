@@ -97,6 +97,10 @@ WORKLOADS = {
     # 63-frame list is gathered into a window before the 720p attention.
     "bounded": Workload("bounded", n_text=512, frames=30, grid_h=23, grid_w=40,
                         cache_frames=240, t0=240, select_frames=63),
+    # the other reading of the bounded history: all 30 frames of the first
+    # segment plus the last 60 cached frames (90 frames, 82,800 tokens)
+    "bounded90": Workload("bounded90", n_text=512, frames=30, grid_h=23, grid_w=40,
+                          cache_frames=240, t0=240, select_frames=90),
 }
 # Full segment sweep: 54 layers x 8 denoising steps of the 720p workload.
 SWEEP_LAYERS = 54

@@ -180,14 +180,15 @@ def test_layer_step_720p_sampled_rows():
 
 
 @pytest.mark.slow
-def test_layer_step_bounded_sampled_rows():
-    w = WORKLOADS["bounded"]
+@pytest.mark.parametrize("name", ["bounded", "bounded90"])
+def test_layer_step_bounded_sampled_rows(name):
+    w = WORKLOADS[name]
     inp, idx, o, lse = _layer_step(w, seed=3, select=True)
     rows = _sample_rows(w, seed=1)
     o_ref, l_ref = _oracle_step(w, inp, idx, rows)
-    assert_close(f64(o[torch.as_tensor(rows)]), o_ref, what="bounded O")
+    assert_close(f64(o[torch.as_tensor(rows)]), o_ref, what=f"{name} O")
     got_l = lse.view(16, -1)[:, torch.as_tensor(rows).cuda()].cpu().numpy().astype(np.float64)
-    assert_close(got_l, l_ref, what="bounded LSE")
+    assert_close(got_l, l_ref, what=f"{name} LSE")
 
 
 def test_wait_timeout_is_reported_and_context_survives():
