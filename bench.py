@@ -399,10 +399,13 @@ def max_over_ranks(values, world: int, device):
 
 def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
     """Times the fp64 oracle (RoPE of sampled query rows + their attention over
-    every key of the workload) on host cores; returns (TFLOP/s, rows, s, threads).
+    every key of the workload) on host cores; returns (TFLOP/s, rows, s,
+    threads, parity).
 
     The oracle works from the seeded inputs (host copies of the resident
-    cache, the frame list and the segment), never from kernel outputs."""
+    cache, the frame list and the segment), never from kernel outputs.  The
+    sampled rows of the step's last output are then compared with the
+    oracle's (`parity`: max and mean absolute error of O and LSE)."""
     import numpy as np
     import torch
 
@@ -424,16 +427,26 @@ def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
     q_all = step.q
     rng = np.random.default_rng(0)
     done, elapsed = 0, 0.0
+    refs = []
     t0 = time.perf_counter()
     while elapsed < budget_s and done < max_rows:
         rows = np.sort(rng.integers(0, ns, rows_per_chunk))
         q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
                                ww[rows])
-        oracle.attention(q_rows, spans)
+        refs.append((rows, oracle.attention(q_rows, spans)))
         done += rows.size
         elapsed = time.perf_counter() - t0
     flops = 4.0 * done * w.n_k * 128 * 16
-    return flops / elapsed / 1e12, done, elapsed, blas_threads()
+    # parity of the step's output on the sampled rows (outside the timing)
+    err_o = np.concatenate([np.abs(f64(step.o[torch.as_tensor(r)]) - o).ravel()
+                            for r, (o, _) in refs])
+    lse_gpu = step.lse.view(16, w.n_q).cpu().numpy().astype(np.float64)
+    err_l = np.concatenate([np.abs(lse_gpu[:, r] - lse).ravel() for r, (_, lse) in refs])
+    parity = {"rows": done, "max_abs_o": float(err_o.max()), "mean_abs_o": float(err_o.mean()),
+              "max_abs_lse": float(err_l.max()), "bar_max_abs": 2e-2, "bar_mean_abs": 2e-3}
+    parity["pass"] = bool(parity["max_abs_o"] <= 2e-2 and parity["mean_abs_o"] <= 2e-3
+                          and parity["max_abs_lse"] <= 2e-2)
+    return flops / elapsed / 1e12, done, elapsed, blas_threads(), parity
 
 
 def blas_threads() -> int:
@@ -566,12 +579,15 @@ def main():
                "overlap": "double-buffered inputs/outputs, separate H2D and D2H streams"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload != "sweep":
-        rate, rows, secs, threads = cpu_oracle_rate(step, budget_s=12.0, rows_per_chunk=16,
-                                                    max_rows=512)
+    parity = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(step, LayerStep):
+        rate, rows, secs, threads, parity = cpu_oracle_rate(step, budget_s=12.0,
+                                                            rows_per_chunk=16, max_rows=512)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"fp64 oracle RoPE + attention of {rows} sampled segment query rows "
                          f"x 16 heads over all {step.w.n_k} keys ({secs:.1f} s)"}
+        if step.sparse is not None:
+            parity = None  # the oracle above is dense attention
 
     if world > 1:
         dist.destroy_process_group()
@@ -605,7 +621,7 @@ def main():
                      "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 burst",
                      "traffic": recorded_traffic(args.workload)},
-        "cpu_baseline": cpu, "e2e": e2e,
+        "cpu_baseline": cpu, "e2e": e2e, "parity": parity,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
     }

@@ -11,6 +11,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "nomas.h"
 #include "nomas_internal.h"
 
@@ -38,6 +40,15 @@ nomas_status ok() {
   g_last_error.clear();
   return NOMAS_OK;
 }
+
+// NVTX range over one C-ABI call (header-only NVTX v3: inert unless a
+// profiler is attached), so that traces show which call enqueued which work.
+struct ApiRange {
+  explicit ApiRange(const char *name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange &) = delete;
+  ApiRange &operator=(const ApiRange &) = delete;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -329,6 +340,7 @@ const char *nomas_version(void) { return "nomas 0.1.0 (sm_100a)"; }
 nomas_status nomas_rope3d_qk(const void *q, const void *k, void *q_out, void *k_out,
                              const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
                              int32_t heads, int32_t head_dim, void *stream) {
+  const ApiRange nvtx_range("nomas_rope3d_qk");
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   int64_t n_video = 0;
@@ -369,6 +381,7 @@ nomas_status nomas_kvcache_append(nomas_kvcache *cache, const void *k_seg, const
                                   int64_t n_tokens, const void *q_in, void *q_out,
                                   const nomas_seg_layout *layout, const nomas_rope3d_cfg *cfg,
                                   void *stream) {
+  const ApiRange nvtx_range("nomas_kvcache_append");
   if (cache == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "cache is NULL");
   CacheView view{cache->k, cache->v, nullptr, nullptr, cache->capacity, cache->len,
                  cache->heads, cache->head_dim, false};
@@ -383,6 +396,7 @@ nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
                                      const void *v_seg, int64_t n_tokens, const void *q_in,
                                      void *q_out, const nomas_seg_layout *layout,
                                      const nomas_rope3d_cfg *cfg, void *stream) {
+  const ApiRange nvtx_range("nomas_kvcache_append_i8");
   if (cache == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "cache is NULL");
   CacheView view{cache->k, cache->v, cache->k_scale, cache->v_scale, cache->capacity,
                  cache->len, cache->heads, cache->head_dim, true};
@@ -396,6 +410,7 @@ nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
 nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame_idx,
                                   int32_t n_frames, int32_t idx_on_device, nomas_kvcache *window,
                                   int32_t *dev_err, void *stream) {
+  const ApiRange nvtx_range("nomas_kvcache_select");
   if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
   CacheView view{src->k, src->v, nullptr, nullptr, src->capacity, src->len,
                  src->heads, src->head_dim, false};
@@ -406,6 +421,7 @@ nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame
 nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
                                      int32_t n_frames, int32_t idx_on_device,
                                      nomas_kvcache *window, int32_t *dev_err, void *stream) {
+  const ApiRange nvtx_range("nomas_kvcache_select_i8");
   if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
   CacheView view{src->k, src->v, src->k_scale, src->v_scale, src->capacity, src->len,
                  src->heads, src->head_dim, true};
@@ -416,6 +432,7 @@ nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t 
 nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,
                                    int64_t n_q, void *o, float *lse, int32_t heads,
                                    int32_t head_dim, void *stream) {
+  const ApiRange nvtx_range("nomas_attention_merge");
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   if (n_parts <= 0 || n_q < 0 || n_q > 0x7fff0000LL)
@@ -452,6 +469,7 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
                                         int32_t n_spans, void *o, float *lse, float softmax_scale,
                                         int32_t heads, int32_t head_dim, int32_t *dev_err,
                                         const nomas_attention_opts *opts, void *stream) {
+  const ApiRange nvtx_range("nomas_segment_attention_ex");
   return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
                           heads, head_dim, dev_err, opts, stream);
 }
@@ -462,6 +480,7 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
                                             int32_t max_tiles, void *o, float *lse,
                                             float softmax_scale, int32_t heads, int32_t head_dim,
                                             int32_t *dev_err, void *stream) {
+  const ApiRange nvtx_range("nomas_segment_attention_sparse");
   if (tile_list == nullptr || tile_count == nullptr)
     return fail(NOMAS_ERR_INVALID_ARG, "tile_list and tile_count are required");
   if (max_tiles < 0) return fail(NOMAS_ERR_INVALID_ARG, "max_tiles < 0");
