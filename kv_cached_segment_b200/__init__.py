@@ -6,8 +6,21 @@ device memory and streams.  There is no CPU fallback: if the compiled
 library is missing, importing the binding's entry points raises.
 
 Entry points (same names as the C ABI, without the ``nomas_`` prefix):
-``rope3d_qk``, ``kvcache_append``, ``kvcache_select``, ``segment_attention``,
-plus the ``KVCache`` holder and the ``RopeConfig`` / ``SegLayout`` structs.
+
+- ``rope3d_qk``: 3D RoPE of a segment's Q (and K) rows;
+- ``kvcache_append`` / ``kvcache_append_i8``: rotate the segment's K into a
+  bf16 or INT8 cache (V copied or quantised), optionally Q too;
+- ``kvcache_select``: gather latent frames of a bf16 or INT8 cache into a
+  bf16 window;
+- ``segment_attention`` / ``segment_attention_sparse``: attention of the
+  query rows over up to four key/value spans, all tiles or listed tiles;
+- ``attention_merge``: combine partial (O, LSE) over disjoint key shards;
+- ``temporal_context_frames``: the power-spaced history frame picker (host).
+
+Holders: ``KVCache`` and ``KVCacheI8`` (caller-owned device buffers plus
+``len``), ``RopeConfig`` and ``SegLayout``.  ``sharded_segment_attention``
+runs key-sharded attention over the ranks of a ``torch.distributed`` group
+(partial attention per rank, all-gather of the partials, merge).
 """
 from __future__ import annotations
 
