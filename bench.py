@@ -54,6 +54,9 @@ def parse_args():
                    help="split the key sequence into this many contiguous shards, attend over "
                         "each into a partial (O, LSE) and merge them (the per-GPU work of "
                         "key-sharded attention, on one GPU); 0 = one launch over all keys")
+    p.add_argument("--kv-splits", default="1",
+                   help="key splits of the attention launch (an integer, or 'auto': chosen from "
+                        "the grid's wave count); 1 = one CTA per query block and head")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -176,6 +179,7 @@ class LayerStep:
         self.launches_per_step = 3 if self.frames else 2
         self.sparse = None
         self.shards = 0
+        self.kv_splits = 1
 
     def use_key_shards(self, n_shards: int):
         """Attention over `n_shards` contiguous ranges of the key sequence
@@ -259,7 +263,8 @@ class LayerStep:
                 mev[1].record()
                 self.merge_ev.append(mev)
         else:
-            nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
+            nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err,
+                                 kv_splits=self.kv_splits)
         if ev is not None:
             ev[1].record()
 
@@ -469,6 +474,17 @@ def make_step(args, rank):
         if args.sparse > 0:
             raise SystemExit("--key-shards and --sparse are exclusive")
         step.use_key_shards(args.key_shards)
+    if args.kv_splits != "1":
+        if not isinstance(step, LayerStep) or step.sparse is not None or step.shards:
+            raise SystemExit("--kv-splits applies to the dense bf16 layer-step only")
+        step.kv_splits = args.kv_splits if args.kv_splits == "auto" else int(args.kv_splits)
+        if step.kv_splits == "auto":
+            w = step.w
+            hist = w.n_window if w.select_frames else w.n_cache
+            step.kv_splits = step.nm.auto_kv_splits(
+                w.n_q, [hist, w.n_text, w.n_seg],
+                step.torch.cuda.get_device_properties(0).multi_processor_count)
+        step.launches_per_step += 1 if step.kv_splits > 1 else 0  # the merge
     return step
 
 
@@ -480,6 +496,8 @@ def workload_text(args, step) -> str:
                 f"{w.n_cache} cached tokens per layer)")
     hist = w.n_window if w.select_frames else w.n_cache
     extra = " (INT8 history cache)" if args.int8 else ""
+    if getattr(step, "kv_splits", 1) > 1:
+        extra += f" (keys split {step.kv_splits} ways per query block, partials merged)"
     if getattr(args, "key_shards", 0) > 0:
         extra += (f" (keys split into {args.key_shards} contiguous shards, partial results "
                   f"merged)")

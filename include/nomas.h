@@ -299,6 +299,38 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
                                             int32_t *dev_err, void *stream);
 
 /*
+ * Key-split attention: the attention of nomas_segment_attention ("How one
+ * segment is made": joint attention of the segment and text over the cached
+ * history and themselves), for shapes whose query blocks alone do not fill
+ * the GPU.  How the keys are cut is this library's choice, not the page's:
+ * the concatenated key tiles (128 keys each, spans in order) are split into
+ * kv_splits contiguous ranges; each (256-row query block, head, range) is one
+ * CTA that writes a partial O (bf16) and LSE into `scratch`, and one merge
+ * (the kernel of nomas_attention_merge) combines them into o and lse.  The
+ * result equals nomas_segment_attention's up to the rounding of the partial
+ * outputs to bf16.
+ *   kv_splits : 1 <= kv_splits <= NOMAS_MAX_MERGE_PARTS; 1 is exactly
+ *               nomas_segment_attention (scratch unused, may be NULL).
+ *   scratch   : caller-owned device memory of at least
+ *               nomas_segment_attention_scratch_bytes(n_q, kv_splits) bytes,
+ *               16-byte aligned, overlapping none of q, o, lse and the spans;
+ *               its contents are overwritten.
+ * Other arguments as nomas_segment_attention.  Errors: as that call, plus
+ * NOMAS_ERR_INVALID_ARG (kv_splits out of range, scratch NULL, misaligned or
+ * overlapping) and NOMAS_ERR_CAPACITY (scratch_bytes too small).
+ */
+nomas_status nomas_segment_attention_split(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                           int32_t n_spans, void *o, float *lse,
+                                           float softmax_scale, int32_t heads, int32_t head_dim,
+                                           int32_t kv_splits, void *scratch,
+                                           int64_t scratch_bytes, int32_t *dev_err,
+                                           void *stream);
+
+/* Scratch bytes nomas_segment_attention_split needs: kv_splits x n_q x
+ * (4096 + 64) for kv_splits > 1 (partial O rows and LSEs), else 0. */
+int64_t nomas_segment_attention_scratch_bytes(int64_t n_q, int32_t kv_splits);
+
+/*
  * Merge of attention results over disjoint key shards ("What 'world memory'
  * stores": the standard preset spreads the cache over eight GPUs, sp_size 8;
  * each GPU attends over its shard and the partial results are combined):

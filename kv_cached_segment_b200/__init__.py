@@ -59,6 +59,8 @@ EXPORTED_SYMBOLS = (
     "nomas_kvcache_select_i8",
     "nomas_segment_attention_sparse",
     "nomas_attention_merge",
+    "nomas_segment_attention_split",
+    "nomas_segment_attention_scratch_bytes",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -151,6 +153,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
                                                    P, P, F32, I32, I32, P, P]
     lib.nomas_attention_merge.restype = ctypes.c_int
     lib.nomas_attention_merge.argtypes = [P, P, I32, I64, P, P, I32, I32, P]
+    lib.nomas_segment_attention_split.restype = ctypes.c_int
+    lib.nomas_segment_attention_split.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, P, P, F32,
+                                                  I32, I32, I32, P, I64, P, P]
+    lib.nomas_segment_attention_scratch_bytes.restype = I64
+    lib.nomas_segment_attention_scratch_bytes.argtypes = [I64, I32]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -375,12 +382,41 @@ def kvcache_select(src, frame_idx, window: KVCache, dev_err=None, stream=None) -
     del keep
 
 
+def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8) -> int:
+    """Key splits for ``segment_attention(kv_splits="auto")``.
+
+    Minimises a simple time model of the launch, in units of one CTA's time
+    per 128-key tile: ceil(CTAs x S / SMs) waves, each as long as one CTA's
+    share of the tiles plus about 3 tiles of fixed cost, plus the merge of
+    the S partial rows (read at ~5.5 TB/s, one tile taking ~1.5 us).  A
+    split must leave at least 4 tiles per CTA and gain at least 2%."""
+    tiles = sum((int(n) + 127) // 128 for n in span_lens)
+    ctas = (int(n_q) + 255) // 256 * HEADS
+    if tiles == 0 or ctas == 0:
+        return 1
+    best, best_t = 1, None
+    for s in range(1, max_splits + 1):
+        if tiles / s < 4:
+            break
+        t = -(-ctas * s // sm_count) * (tiles / s + 3.0)
+        if s > 1:
+            t += (s + 1) * n_q * (16 * 128 * 2 + 16 * 4) / 5.5e12 / 1.5e-6 + 3.0
+        if best_t is None or t < 0.98 * best_t:
+            best, best_t = s, t
+    return best
+
+
 def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, dev_err=None,
-                      stream=None, wait_limit_ns: int = 0, testing_skip_kv_load: int = -1):
+                      stream=None, wait_limit_ns: int = 0, testing_skip_kv_load: int = -1,
+                      kv_splits=1):
     """Attention of every row of q over all keys of ``spans`` (list of (k, v)); returns o.
 
     ``wait_limit_ns`` bounds every pipeline wait in the kernel (0: default);
     ``testing_skip_kv_load`` is for tests of the timeout path only.
+    ``kv_splits`` > 1 (or "auto", see ``auto_kv_splits``) cuts the key tiles
+    into that many ranges computed by separate CTAs and merged, for shapes
+    whose query blocks alone do not fill the GPU; the scratch for the
+    partial results is allocated here, through PyTorch.
     """
     lib = load_library()
     n_q = _rows(q, "q")
@@ -400,7 +436,26 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
     if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
         raise TypeError("dev_err must be a CUDA int32 tensor")
-    if wait_limit_ns or testing_skip_kv_load != -1:
+    if kv_splits == "auto":
+        sm = torch.cuda.get_device_properties(q.device).multi_processor_count
+        kv_splits = auto_kv_splits(n_q, [int(k.shape[0]) for k, _ in spans], sm)
+    kv_splits = int(kv_splits)
+    if kv_splits > 1:
+        if wait_limit_ns or testing_skip_kv_load != -1:
+            raise ValueError("kv_splits > 1 takes no wait_limit_ns / testing_skip_kv_load")
+        if stream is not None and not isinstance(stream, torch.cuda.Stream):
+            raise TypeError("kv_splits > 1 takes stream=None or a torch.cuda.Stream")
+        nbytes = lib.nomas_segment_attention_scratch_bytes(n_q, kv_splits)
+        scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        _check(lib.nomas_segment_attention_split(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
+                                                 float(softmax_scale), HEADS, HEAD_DIM, kv_splits,
+                                                 _ptr(scratch), nbytes, _ptr(dev_err),
+                                                 _stream(stream)))
+        # allocated on the current stream; when the kernels run on another
+        # one, the allocator must not hand the scratch out before they end
+        if stream is not None:
+            scratch.record_stream(stream)
+    elif wait_limit_ns or testing_skip_kv_load != -1:
         opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load))
         _check(lib.nomas_segment_attention_ex(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
                                               float(softmax_scale), HEADS, HEAD_DIM,

@@ -327,7 +327,15 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               int32_t n_spans, const int32_t *tile_list,
                               const int32_t *tile_count, int32_t max_tiles, void *o, float *lse,
                               float softmax_scale, int32_t heads, int32_t head_dim,
-                              int32_t *dev_err, const nomas_attention_opts *opts, void *stream);
+                              int32_t *dev_err, const nomas_attention_opts *opts,
+                              int32_t kv_splits, void *scratch, int64_t scratch_bytes,
+                              void *stream);
+
+// Scratch of a key-split attention: S partial outputs [S][n_q][16][128] bf16,
+// then their LSEs [S][16][n_q] fp32.
+int64_t split_scratch_bytes(int64_t n_q, int32_t kv_splits) {
+  return (int64_t)kv_splits * n_q * (kRowBytes + kHeads * 4);
+}
 
 }  // namespace
 
@@ -471,7 +479,24 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
                                         const nomas_attention_opts *opts, void *stream) {
   const ApiRange nvtx_range("nomas_segment_attention_ex");
   return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
-                          heads, head_dim, dev_err, opts, stream);
+                          heads, head_dim, dev_err, opts, 1, nullptr, 0, stream);
+}
+
+int64_t nomas_segment_attention_scratch_bytes(int64_t n_q, int32_t kv_splits) {
+  if (n_q < 0 || kv_splits < 1) return 0;
+  return kv_splits > 1 ? split_scratch_bytes(n_q, kv_splits) : 0;
+}
+
+nomas_status nomas_segment_attention_split(const void *q, int64_t n_q, const nomas_kv_span *spans,
+                                           int32_t n_spans, void *o, float *lse,
+                                           float softmax_scale, int32_t heads, int32_t head_dim,
+                                           int32_t kv_splits, void *scratch,
+                                           int64_t scratch_bytes, int32_t *dev_err,
+                                           void *stream) {
+  const ApiRange nvtx_range("nomas_segment_attention_split");
+  return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
+                          heads, head_dim, dev_err, nullptr, kv_splits, scratch, scratch_bytes,
+                          stream);
 }
 
 nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
@@ -489,7 +514,8 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
   if ((reinterpret_cast<uintptr_t>(tile_list) & 3u) || (reinterpret_cast<uintptr_t>(tile_count) & 3u))
     return fail(NOMAS_ERR_INVALID_ARG, "tile_list and tile_count must be 4-byte aligned");
   return attention_common(q, n_q, spans, n_spans, tile_list, tile_count, max_tiles, o, lse,
-                          softmax_scale, heads, head_dim, dev_err, nullptr, stream);
+                          softmax_scale, heads, head_dim, dev_err, nullptr, 1, nullptr, 0,
+                          stream);
 }
 
 }  // extern "C"
@@ -500,9 +526,14 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               int32_t n_spans, const int32_t *tile_list,
                               const int32_t *tile_count, int32_t max_tiles, void *o, float *lse,
                               float softmax_scale, int32_t heads, int32_t head_dim,
-                              int32_t *dev_err, const nomas_attention_opts *opts, void *stream) {
+                              int32_t *dev_err, const nomas_attention_opts *opts,
+                              int32_t kv_splits, void *scratch, int64_t scratch_bytes,
+                              void *stream) {
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
+  if (kv_splits < 1 || kv_splits > NOMAS_MAX_MERGE_PARTS)
+    return fail(NOMAS_ERR_INVALID_ARG, "kv_splits must be in [1, %d] (got %d)",
+                NOMAS_MAX_MERGE_PARTS, kv_splits);
   if (n_spans < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_spans < 0");
   if (n_spans > kMaxSpans)
     return fail(NOMAS_ERR_UNSUPPORTED, "at most %d key/value spans (got %d)", kMaxSpans, n_spans);
@@ -518,6 +549,17 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   if (overlap(q, qb, o, qb)) return fail(NOMAS_ERR_INVALID_ARG, "o overlaps q");
   if (lse != nullptr && (overlap(lse, n_q * kHeads * 4, o, qb) || overlap(lse, n_q * kHeads * 4, q, qb)))
     return fail(NOMAS_ERR_INVALID_ARG, "lse overlaps q or o");
+  const int64_t sb = kv_splits > 1 ? split_scratch_bytes(n_q, kv_splits) : 0;
+  if (kv_splits > 1) {
+    if (scratch == nullptr || !aligned16(scratch))
+      return fail(NOMAS_ERR_INVALID_ARG, "scratch must be non-NULL and 16-byte aligned");
+    if (scratch_bytes < sb)
+      return fail(NOMAS_ERR_CAPACITY, "scratch of %lld bytes, %lld needed", (long long)scratch_bytes,
+                  (long long)sb);
+    if (overlap(scratch, sb, q, qb) || overlap(scratch, sb, o, qb) ||
+        (lse != nullptr && overlap(scratch, sb, lse, n_q * kHeads * 4)))
+      return fail(NOMAS_ERR_INVALID_ARG, "scratch overlaps q, o or lse");
+  }
   AttnArgs a{};
   int n_used = 0;
   for (int s = 0; s < n_spans; ++s) {
@@ -530,8 +572,9 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
     const int64_t sbytes = sp.len * kRowBytes;
     if (overlap(sp.k, sbytes, o, qb) || overlap(sp.v, sbytes, o, qb) ||
         (lse != nullptr && (overlap(sp.k, sbytes, lse, n_q * kHeads * 4) ||
-                            overlap(sp.v, sbytes, lse, n_q * kHeads * 4))))
-      return fail(NOMAS_ERR_INVALID_ARG, "span %d overlaps an output", s);
+                            overlap(sp.v, sbytes, lse, n_q * kHeads * 4))) ||
+        overlap(sp.k, sbytes, scratch, sb) || overlap(sp.v, sbytes, scratch, sb))
+      return fail(NOMAS_ERR_INVALID_ARG, "span %d overlaps an output or the scratch", s);
     if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len)) != NOMAS_OK) return st;
     if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len)) != NOMAS_OK) return st;
     a.span_len[n_used] = sp.len;
@@ -554,6 +597,19 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   a.n_q = (int32_t)n_q;
   a.o = static_cast<uint16_t *>(o);
   a.lse = lse;
+  a.kv_splits = 1;
+  uint16_t *part_o = nullptr;
+  float *part_lse = nullptr;
+  if (kv_splits > 1) {
+    // Partial results of the S key ranges go to the scratch, then one merge
+    // writes o and lse.
+    part_o = static_cast<uint16_t *>(scratch);
+    part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) +
+                                         (int64_t)kv_splits * n_q * kRowBytes);
+    a.o = part_o;
+    a.lse = part_lse;
+    a.kv_splits = kv_splits;
+  }
   a.dev_err = dev_err;
   a.wait_limit_ns = g_wait_limit_ns;
   a.testing_skip_load = -1;
@@ -563,8 +619,13 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
       return fail(NOMAS_ERR_INVALID_ARG, "testing_skip_kv_load must be >= -1");
     a.testing_skip_load = opts->testing_skip_kv_load;
   }
-  const cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  if (kv_splits > 1) {
+    e = launch_merge(part_o, part_lse, kv_splits, n_q, static_cast<uint16_t *>(o), lse,
+                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "merge of key splits launch");
+  }
   return ok();
 }
 

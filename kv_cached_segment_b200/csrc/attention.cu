@@ -325,7 +325,8 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
 __device__ __forceinline__ int num_tiles(int64_t len) { return (int)((len + kBN - 1) / kBN); }
 
 // Walks this block's key tiles as (span, tile within the span).  Dense mode
-// visits every tile of every span in order with two counters; sparse mode
+// visits the global tiles [g0, g1) in order (all of them without a key
+// split); sparse mode
 // reads the block's list of global tile ids (tiles numbered across the
 // concatenated spans) and skips ids outside the spans -- every role walks the
 // same list the same way, so they agree on the sequence.
@@ -334,8 +335,16 @@ struct TileWalk {
   const AttnArgs &p;
   const int32_t *list;
   int n_list;
-  int idx = 0, s = 0, kt = 0;
-  __device__ TileWalk(const AttnArgs &a, const int32_t *l, int n) : p(a), list(l), n_list(n) {}
+  int idx = 0, s = 0, kt = 0, g = 0, g_end = 0;
+  __device__ TileWalk(const AttnArgs &a, const int32_t *l, int n, int g0, int g1)
+      : p(a), list(l), n_list(n) {
+    if constexpr (!kSparse) {
+      g = g0;
+      g_end = g1;
+      while (s + 1 < p.n_spans && g0 >= p.tile_base[s + 1]) ++s;
+      kt = g0 - p.tile_base[s];
+    }
+  }
   // Next tile; false at the end.  `bad` is set when an invalid id was skipped.
   __device__ __forceinline__ bool next(int *span, int *ktile, bool *bad) {
     if constexpr (kSparse) {
@@ -353,13 +362,14 @@ struct TileWalk {
       }
       return false;
     } else {
-      while (s < p.n_spans && kt >= num_tiles(p.span_len[s])) {
+      if (g >= g_end) return false;
+      *span = s;
+      *ktile = kt;
+      ++g;
+      if (++kt >= p.tile_base[s + 1] - p.tile_base[s]) {
         ++s;
         kt = 0;
       }
-      if (s >= p.n_spans) return false;
-      *span = s;
-      *ktile = kt++;
       return true;
     }
   }
@@ -416,13 +426,18 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
   // This block's key tiles: the whole key sequence, or its sparse list.
   const int32_t *list = nullptr;
   int n_list = 0;
-  int n_kv = p.tile_base[p.n_spans];  // K/V tiles this block streams
+  // Dense: this block's share [g0, g1) of the key tiles (all of them unless
+  // the keys are split across the grid's third dimension).
+  const int total_tiles = p.tile_base[p.n_spans];
+  const int g0 = (int)((int64_t)total_tiles * blockIdx.z / p.kv_splits);
+  const int g1 = (int)((int64_t)total_tiles * (blockIdx.z + 1) / p.kv_splits);
+  int n_kv = g1 - g0;  // K/V tiles this block streams
   if constexpr (kSparse) {
     const int64_t row = (int64_t)blockIdx.x * kHeads + head;
     list = p.tile_list + row * p.max_tiles;
     n_list = min(max(p.tile_count[row], 0), p.max_tiles);
     n_kv = 0;
-    TileWalk<true> w(p, list, n_list);
+    TileWalk<true> w(p, list, n_list, 0, 0);
     int s_, kt_;
     bool bad_ = false;
     while (w.next(&s_, &kt_, &bad_)) ++n_kv;
@@ -440,7 +455,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
                       head * kHeadDim + c * 64, q_row0 + i * kBM, pol_q);
       int t = 0;
       bool ok = true;
-      TileWalk<kSparse> walk(p, list, n_list);
+      TileWalk<kSparse> walk(p, list, n_list, g0, g1);
       int s, kt;
       bool bad = false;
       while (ok && walk.next(&s, &kt, &bad)) {
@@ -546,7 +561,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
     float l = 0.f;        // running row sum of exp2(...)
     bool ok = true;
     int j = 0;
-    TileWalk<kSparse> walk(p, list, n_list);
+    TileWalk<kSparse> walk(p, list, n_list, g0, g1);
     int s, kt;
     bool bad = false;
     while (ok && walk.next(&s, &kt, &bad)) {
@@ -703,14 +718,18 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
         ++j;
       }
     }
-    // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l).
+    // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l), into part
+    // blockIdx.z of the outputs when the keys are split.
+    uint16_t *const o_out = p.o + (int64_t)blockIdx.z * p.n_q * kRowElems;
+    float *const lse_out =
+        p.lse == nullptr ? nullptr : p.lse + (int64_t)blockIdx.z * kHeads * p.n_q;
     bool have_o = ok && n_kv > 0;
     if (have_o) have_o = __all_sync(0xffffffffu, wait_phase(bar(kBarOFull + tile), 0, ctl));
     if (have_o) {
       tc_fence_after();
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       const float inv_l = 1.0f / l;
-      uint16_t *orow_g = p.o + row * kRowElems + head * kHeadDim;
+      uint16_t *orow_g = o_out + row * kRowElems + head * kHeadDim;
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t orow[32];
@@ -729,17 +748,17 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           }
         }
       }
-      if (p.lse != nullptr && row < p.n_q)
-        p.lse[(int64_t)head * p.n_q + row] = (m + log2f(l)) * 0.69314718055994531f;
+      if (lse_out != nullptr && row < p.n_q)
+        lse_out[(int64_t)head * p.n_q + row] = (m + log2f(l)) * 0.69314718055994531f;
     } else if (ok && n_kv == 0) {
       // No key selected for this block (a sparse list with no valid entry):
       // the empty sums give O = 0 and LSE = -inf.
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       if (row < p.n_q) {
-        uint4 *dst = reinterpret_cast<uint4 *>(p.o + row * kRowElems + head * kHeadDim);
+        uint4 *dst = reinterpret_cast<uint4 *>(o_out + row * kRowElems + head * kHeadDim);
 #pragma unroll
         for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-        if (p.lse != nullptr) p.lse[(int64_t)head * p.n_q + row] = -INFINITY;
+        if (lse_out != nullptr) lse_out[(int64_t)head * p.n_q + row] = -INFINITY;
       }
     }
   }
@@ -785,7 +804,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   const int64_t q_blocks = ((int64_t)a.n_q + kQTiles * kBM - 1) / (kQTiles * kBM);
   if (q_blocks <= 0) return cudaSuccess;
   if (q_blocks > 0x7fffffff) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)q_blocks, kHeads);
+  if (a.kv_splits < 1 || a.kv_splits > NOMAS_MAX_MERGE_PARTS ||
+      (a.kv_splits > 1 && (a.tile_list != nullptr || a.lse == nullptr)))
+    return cudaErrorInvalidValue;
+  dim3 grid((unsigned)q_blocks, kHeads, (unsigned)a.kv_splits);
   if (a.tile_list != nullptr)
     attention_kernel<true><<<grid, kThreads, kSmemAlloc, stream>>>(a);
   else

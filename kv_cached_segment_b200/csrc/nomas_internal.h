@@ -91,6 +91,11 @@ struct AttnArgs {
   const int32_t *tile_count;   // [q_blocks][heads] entries used in each row
   int32_t max_tiles;
   int32_t tile_base[kMaxSpans + 1];  // first global tile id of each span; [n_spans] = total
+  // Split of the key tiles (dense mode): block z of the grid's third
+  // dimension streams global tiles [T z / S, T (z + 1) / S) of the T tiles and
+  // writes its partial O and LSE to part z of o ([S][n_q][16][128]) and lse
+  // ([S][16][n_q]).  1: no split.
+  int32_t kv_splits;
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,

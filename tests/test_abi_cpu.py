@@ -258,3 +258,27 @@ def test_merge_validation(lib):
     assert f(parts, lse_parts, 4, 100, o, lse_parts, 16, 128, None) \
         == nm.NOMAS_ERR_INVALID_ARG  # merged LSE over the partial LSEs
     assert f(parts, lse_parts, 4, 0, None, None, 16, 128, None) == nm.NOMAS_OK  # nothing to do
+
+
+def test_split_attention_validation_and_scratch_size(lib):
+    assert lib.nomas_segment_attention_scratch_bytes(1000, 1) == 0
+    assert lib.nomas_segment_attention_scratch_bytes(1000, 3) == 3 * 1000 * (ROW + 64)
+    spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, 1000))
+    o, lse, scr = FAKE + 3 * 10 ** 9, FAKE + 4 * 10 ** 9, FAKE + 5 * 10 ** 9
+    need = 4 * 100 * (ROW + 64)
+    f = lib.nomas_segment_attention_split
+    for splits in (0, nm.MAX_MERGE_PARTS + 1):
+        assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, splits, scr, need, None, None) \
+            == nm.NOMAS_ERR_INVALID_ARG
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, 4, None, need, None, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # no scratch
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, 4, scr + 8, need, None, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # misaligned scratch
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, 4, scr, need - 1, None, None) \
+        == nm.NOMAS_ERR_CAPACITY
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, 4, o - 4096, need, None, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # scratch overlaps o
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 128, 4, FAKE + 10 ** 9, need, None, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # scratch overlaps a span
+    assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 64, 4, scr, need, None, None) \
+        == nm.NOMAS_ERR_UNSUPPORTED

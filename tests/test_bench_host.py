@@ -33,3 +33,22 @@ def test_key_shards_cover_the_key_sequence_once_in_order(shards):
     assert all(f % 128 == 0 for f in firsts)
     if shards > (sum(lens) + 127) // 128:
         assert any(sub[0][0].numel() == 0 for sub in parts)
+
+
+def test_auto_kv_splits_fills_the_gpu_only_when_it_pays():
+    from seeded_inputs import WORKLOADS
+
+    def splits(name):
+        w = WORKLOADS[name]
+        hist = w.n_window if w.select_frames else w.n_cache
+        return nm.auto_kv_splits(w.n_q, [hist, w.n_text, w.n_seg])
+
+    # 11.9 waves of query blocks already: no split; 3.35 waves: split in two
+    assert splits("720p") == 1 and splits("bounded") == 1 and splits("bounded90") == 1
+    assert splits("short") == 2
+    # too few tiles to split
+    assert splits("tiny") == 1
+    # 2 query blocks x 16 heads over 652 key tiles: as many splits as fit one wave
+    s = nm.auto_kv_splits(512, [55200, 512, 27600])
+    assert 32 * s <= 148 and 32 * (s + 1) > 148
+    assert nm.auto_kv_splits(0, [100]) == 1 and nm.auto_kv_splits(100, []) == 1
