@@ -56,6 +56,9 @@ typedef enum {
 #define NOMAS_HEAD_DIM 128
 #define NOMAS_MAX_SPANS 4
 #define NOMAS_MAX_MERGE_PARTS 32 /* partial results one attention merge combines */
+/* Size of the scratch array built into the library for
+ * nomas_segment_attention_split_noalloc: 64 MiB per device that uses it. */
+#define NOMAS_NOALLOC_SCRATCH_BYTES (64ll << 20)
 
 /*
  * 3D rotary configuration: the head dimension is split into a temporal chunk
@@ -329,6 +332,40 @@ nomas_status nomas_segment_attention_split(const void *q, int64_t n_q, const nom
 /* Scratch bytes nomas_segment_attention_split needs: kv_splits x n_q x
  * (4096 + 64) for kv_splits > 1 (partial O rows and LSEs), else 0. */
 int64_t nomas_segment_attention_scratch_bytes(int64_t n_q, int32_t kv_splits);
+
+/*
+ * nomas_segment_attention_split for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call: it exists for this
+ * library's users.  A caller whose device memory is claimed up front (a
+ * serving process with a fixed budget handed out from its own pools), one
+ * inside a framework that owns the device allocator and forbids allocations
+ * behind its back, or one on a latency-critical path where cudaMalloc and
+ * cudaFree (which can synchronise the device) are not allowed, cannot supply
+ * the scratch that nomas_segment_attention_split takes.  This call uses an
+ * array of NOMAS_NOALLOC_SCRATCH_BYTES built into the library instead, and
+ * allocates nothing.
+ *   Arguments as nomas_segment_attention_split, without scratch.
+ *   Limit: kv_splits x n_q x (4096 + 64) bytes must fit in the array
+ *   (about 8,000 query rows with 2 splits); larger requests return
+ *   NOMAS_ERR_CAPACITY with a message giving both sizes, before anything is
+ *   launched.
+ *   The array is held on every device that uses this call until the process
+ *   exits.  The first call on a device looks up the array's device address
+ *   (with that device current) and keeps it: make that first call before any
+ *   stream capture begins.
+ *   Every call shares the array: calls that can run at the same time on the
+ *   GPU (different streams, or different host threads) race on it and must
+ *   be ordered by the caller.  Each call writes every byte of scratch it
+ *   reads, so a call never sees the previous call's contents.
+ * Errors: as nomas_segment_attention_split, plus NOMAS_ERR_CAPACITY (the
+ * request exceeds the array) and NOMAS_ERR_CUDA (the address lookup failed).
+ */
+nomas_status nomas_segment_attention_split_noalloc(const void *q, int64_t n_q,
+                                                   const nomas_kv_span *spans, int32_t n_spans,
+                                                   void *o, float *lse, float softmax_scale,
+                                                   int32_t heads, int32_t head_dim,
+                                                   int32_t kv_splits, int32_t *dev_err,
+                                                   void *stream);
 
 /*
  * Merge of attention results over disjoint key shards ("What 'world memory'

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libnomas.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["abi.cu", "rope_append.cu", "select.cu", "attention.cu", "frame_picker.cu", "merge.cu"]
+SOURCES = ["abi.cu", "rope_append.cu", "select.cu", "attention.cu", "frame_picker.cu", "merge.cu",
+           "noalloc.cu"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3",

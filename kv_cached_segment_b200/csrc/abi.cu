@@ -631,3 +631,8 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
 
 }  // namespace
 
+// Records a failure from another source file of the library in the same
+// per-thread message that nomas_last_error() returns.
+nomas_status nomas::report_error(nomas_status st, const char *message) {
+  return fail(st, "%s", message);
+}

@@ -105,4 +105,8 @@ cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
 cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_t n_parts,
                          int64_t n_q, uint16_t *o, float *lse, cudaStream_t stream);
 
+// ----------------------------------------------------------------- errors --
+// Sets the message nomas_last_error() returns on this thread; returns st.
+nomas_status report_error(nomas_status st, const char *message);
+
 }  // namespace nomas
