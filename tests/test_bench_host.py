@@ -52,3 +52,36 @@ def test_auto_kv_splits_fills_the_gpu_only_when_it_pays():
     s = nm.auto_kv_splits(512, [55200, 512, 27600])
     assert 32 * s <= 148 and 32 * (s + 1) > 148
     assert nm.auto_kv_splits(0, [100]) == 1 and nm.auto_kv_splits(100, []) == 1
+
+
+def test_sparse_tile_lists_keep_spans_whole_and_sample_candidates():
+    from seeded_inputs import sparse_tile_lists
+
+    lens = [1000, 37, 700]                 # 8 + 1 + 6 tiles, global ids 0-7, 8, 9-14
+    lists, counts = sparse_tile_lists(600, lens, keep_spans=[1], candidate_spans=[0, 2],
+                                      fraction=0.25, seed=3)
+    assert lists.shape == (3, 16, 1 + 4) and counts.shape == (3, 16)   # round(0.25 * 14) = 4
+    assert (counts == 5).all()
+    seen = set()
+    for b in range(3):
+        for h in range(16):
+            row = lists[b, h, :counts[b, h]].tolist()
+            assert row == sorted(set(row))                 # sorted, no repeats
+            assert 8 in row                                # the kept span's only tile
+            assert all(0 <= g < 15 for g in row)
+            picked = [g for g in row if g != 8]              # the sampled candidates
+            assert len(picked) == 4 and all(g in range(0, 8) or g in range(9, 15) for g in picked)
+            seen.add(tuple(row))
+    assert len(seen) > 1                                   # blocks and heads differ
+    again, _ = sparse_tile_lists(600, lens, [1], [0, 2], 0.25, seed=3)
+    assert (again == lists).all()                          # seeded: reproducible
+    other, _ = sparse_tile_lists(600, lens, [1], [0, 2], 0.25, seed=4)
+    assert not (other == lists).all()
+
+
+def test_sparse_tile_lists_pad_with_minus_one():
+    from seeded_inputs import sparse_tile_lists
+
+    lists, counts = sparse_tile_lists(100, [300], keep_spans=[], candidate_spans=[0],
+                                      fraction=0.0, seed=1)
+    assert (counts == 0).all() and (lists == -1).all() and lists.shape[-1] == 1
