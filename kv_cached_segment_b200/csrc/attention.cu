@@ -244,13 +244,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-
 // 2^x for a pair of values on the FMA pipe, to share the exponential work of
 // the softmax between the MUFU unit and the FMA units.  Cody-Waite style
 // reduction: adding 1.5 * 2^23 rounds x to the nearest integer j (kept in the
 // low mantissa bits of the sum), f = x - j lies in [-1/2, 1/2] exactly, 2^f
-// comes from a degree-3 polynomial whose coefficients were fitted here by the
-// Remez exchange algorithm to minimise the relative error on [-1/2, 1/2]
+// comes from a degree-3 polynomial whose coefficients were fitted by the
+// Remez exchange algorithm (fit_exp2_poly.py in this package) to minimise the
+// relative error on [-1/2, 1/2]
 // (max 7.5e-5, far below the 2^-9 rounding step of the bf16 P it feeds), and
 // j is added to the exponent field.  x is clamped at -125 so the exponent
 // cannot underflow; 2^-125 stands in for 0.
