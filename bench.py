@@ -23,6 +23,7 @@ import statistics
 import subprocess
 import sys
 import time
+import types
 
 import numpy as np
 
@@ -779,10 +780,19 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: {rows_per_step} sampled segment query rows per step "
-                               f"x 16 heads over all {w.n_k} keys", "n_q": w.n_q, "n_k": w.n_k},
+        # the same workload as the CUDA arm's line; what was sampled is in
+        # cpu_baseline.sample
+        "config": {"workload": workload_text(args, types.SimpleNamespace(w=w, kv_splits=1)),
+                   "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
+                   "attention_flops_per_step": w.attention_flops(),
+                   "step": "fused rope3d+append" + (" + select" if w.select_frames else "")
+                           + " + segment attention",
+                   "l2": "host memory (the oracle runs on the CPU)",
+                   "parallelism": "one process on the host cores"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_per_step} query rows per step, {args.steps} steps"},
+                         "sample": f"fp64 oracle RoPE + attention of {rows_per_step} sampled "
+                                   f"segment query rows per step x 16 heads over all {w.n_k} "
+                                   f"keys, {args.steps} steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
