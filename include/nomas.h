@@ -55,7 +55,8 @@ typedef enum {
 #define NOMAS_HEADS 16
 #define NOMAS_HEAD_DIM 128
 #define NOMAS_MAX_SPANS 4
-#define NOMAS_MAX_MERGE_PARTS 32 /* partial results one attention merge combines */
+#define NOMAS_MAX_MERGE_PARTS 32   /* partial results one attention merge combines */
+#define NOMAS_MAX_MERGE_OUTPUTS 32 /* outputs one peer merge writes its rows to     */
 /* Size of the scratch array built into the library for
  * nomas_segment_attention_split_noalloc: 64 MiB per device that uses it. */
 #define NOMAS_NOALLOC_SCRATCH_BYTES (64ll << 20)
@@ -383,6 +384,37 @@ nomas_status nomas_segment_attention_split_noalloc(const void *q, int64_t n_q,
 nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,
                                    int64_t n_q, void *o, float *lse, int32_t heads,
                                    int32_t head_dim, void *stream);
+
+/*
+ * The merge of key-shard partials fused with their exchange between GPUs
+ * ("What 'world memory' stores": the cache spread over eight GPUs, sp_size 8;
+ * how the partial results meet is not on the page).  Each GPU calls it for
+ * the query rows it owns: it reads those rows of every GPU's partial result
+ * and writes the merged rows into every listed output, so the partials cross
+ * NVLink once, only for the rows the caller merges, and the merged rows are
+ * distributed in the same kernel.  The pointers may address other GPUs'
+ * memory mapped into this process (peer access, CUDA IPC or symmetric
+ * memory); the kernel reads and writes them with plain loads and stores.
+ *   o_parts, lse_parts: host arrays of n_parts device pointers; part r is a
+ *                       [n_q][heads][head_dim] bf16 partial output and its
+ *                       [heads][n_q] fp32 LSE (natural log).
+ *   row0, n_rows      : the query rows merged by this call.
+ *   o_outs, lse_outs  : host arrays of n_outs device pointers to
+ *                       [n_q][heads][head_dim] bf16 outputs and [heads][n_q]
+ *                       fp32 LSEs; rows [row0, row0 + n_rows) of each are
+ *                       written.  lse_outs may be NULL, or hold NULL entries.
+ * 1 <= n_parts <= NOMAS_MAX_MERGE_PARTS, 1 <= n_outs <= NOMAS_MAX_MERGE_OUTPUTS.
+ * The caller orders the call after every producer of the partials, on every
+ * GPU, and every consumer of the outputs after the calls of all GPUs: for
+ * example with a one-element NCCL all-reduce on the same streams before and
+ * after.  Outputs must not overlap the partials.
+ * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
+ */
+nomas_status nomas_attention_merge_peers(const void *const *o_parts, const float *const *lse_parts,
+                                         int32_t n_parts, int64_t n_q, int64_t row0,
+                                         int64_t n_rows, void *const *o_outs,
+                                         float *const *lse_outs, int32_t n_outs, int32_t heads,
+                                         int32_t head_dim, void *stream);
 
 #ifdef __cplusplus
 }

@@ -45,6 +45,7 @@ DEVERR_BAD_FRAME_INDEX = 0x1
 DEVERR_WAIT_TIMEOUT = 0x2
 MAX_SPANS = 4
 MAX_MERGE_PARTS = 32
+MAX_MERGE_OUTPUTS = 32
 
 EXPORTED_SYMBOLS = (
     "nomas_last_error",
@@ -61,6 +62,7 @@ EXPORTED_SYMBOLS = (
     "nomas_attention_merge",
     "nomas_segment_attention_split",
     "nomas_segment_attention_scratch_bytes",
+    "nomas_attention_merge_peers",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -158,6 +160,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
                                                   I32, I32, I32, P, I64, P, P]
     lib.nomas_segment_attention_scratch_bytes.restype = I64
     lib.nomas_segment_attention_scratch_bytes.argtypes = [I64, I32]
+    lib.nomas_attention_merge_peers.restype = ctypes.c_int
+    lib.nomas_attention_merge_peers.argtypes = [P, P, I32, I64, I64, I64, P, P, I32, I32, I32, P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -523,12 +527,64 @@ def attention_merge(o_parts, lse_parts, o=None, lse=None, stream=None):
     return o
 
 
+def attention_merge_peers(o_parts, lse_parts, o_outs, lse_outs=None, row0: int = 0,
+                          n_rows: int | None = None, stream=None):
+    """Merge rows [row0, row0 + n_rows) of key-shard partials found through
+    lists of tensors, writing the merged rows into every tensor of o_outs
+    (and lse_outs).  The tensors may live on other GPUs whose memory this
+    process can reach (peer access, IPC or symmetric memory): the exchange
+    between GPUs and the merge are one kernel.  The caller orders the call
+    after every GPU's partials are complete, and the outputs' readers after
+    every GPU's call.
+
+    o_parts: R bf16 [n_q][16][128]; lse_parts: R fp32 [16][n_q] (or flat);
+    o_outs: bf16 [n_q][16][128] outputs; lse_outs: fp32 LSE outputs or None."""
+    lib = load_library()
+    n_parts, n_outs = len(o_parts), len(o_outs)
+    if len(lse_parts) != n_parts:
+        raise ValueError("o_parts and lse_parts differ in length")
+    n_q = _rows(o_parts[0], "o_parts[0]")
+    for i, t in enumerate(list(o_parts) + list(o_outs)):
+        if _rows(t, f"partial/output {i}") != n_q:
+            raise ValueError("every partial and output must have n_q rows")
+    for t in list(lse_parts) + list(lse_outs or []):
+        if t.dtype != torch.float32 or t.numel() != HEADS * n_q or not t.is_contiguous():
+            raise ValueError("LSE tensors must be contiguous fp32 with heads * n_q elements")
+    if lse_outs is not None and len(lse_outs) != n_outs:
+        raise ValueError("o_outs and lse_outs differ in length")
+    n_rows = n_q - row0 if n_rows is None else n_rows
+    parts = (ctypes.c_void_p * n_parts)(*[t.data_ptr() for t in o_parts])
+    lses = (ctypes.c_void_p * n_parts)(*[t.data_ptr() for t in lse_parts])
+    outs = (ctypes.c_void_p * n_outs)(*[t.data_ptr() for t in o_outs])
+    louts = (ctypes.c_void_p * n_outs)(*[t.data_ptr() for t in lse_outs]) if lse_outs else None
+    _check(lib.nomas_attention_merge_peers(parts, lses, n_parts, n_q, int(row0), int(n_rows), outs,
+                                           louts, n_outs, HEADS, HEAD_DIM, _stream(stream)))
+
+
 def shard_rows(n: int, rank: int, world: int, align: int = 1):
     """Contiguous share [a, b) of n rows for `rank` (boundaries on multiples of align)."""
     units = (n + align - 1) // align
     a = (units * rank) // world * align
     b = min(n, (units * (rank + 1)) // world * align)
     return min(a, n), b
+
+
+def peer_partial_attention(q, local_spans, part_o, part_lse):
+    """Phase 1 of key-sharded attention over peer memory: this GPU's partial
+    (O, LSE) over its own key spans, into its slot of the partial buffers."""
+    segment_attention(q, local_spans, o=part_o, lse=part_lse.view(-1))
+
+
+def peer_merge_owned_rows(part_o_peers, part_lse_peers, o_peers, lse_peers, rank: int,
+                          world: int):
+    """Phase 2: this GPU merges the query rows it owns (a contiguous share,
+    on 16-row boundaries) from every GPU's partial and writes them into every
+    GPU's output.  Between phase 1 on all GPUs and this call, and after this
+    call on all GPUs, the caller needs a cross-GPU barrier in stream order
+    (for example a one-element NCCL all-reduce)."""
+    n_q = part_o_peers[0].shape[0]
+    a, b = shard_rows(n_q, rank, world, align=16)
+    attention_merge_peers(part_o_peers, part_lse_peers, o_peers, lse_peers, row0=a, n_rows=b - a)
 
 
 def sharded_segment_attention(q, local_spans, group=None, lse=None, attend=None, merge=None):

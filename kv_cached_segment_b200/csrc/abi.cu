@@ -465,6 +465,47 @@ nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, 
   return ok();
 }
 
+nomas_status nomas_attention_merge_peers(const void *const *o_parts, const float *const *lse_parts,
+                                         int32_t n_parts, int64_t n_q, int64_t row0,
+                                         int64_t n_rows, void *const *o_outs,
+                                         float *const *lse_outs, int32_t n_outs, int32_t heads,
+                                         int32_t head_dim, void *stream) {
+  const ApiRange nvtx_range("nomas_attention_merge_peers");
+  nomas_status st = check_shape(heads, head_dim);
+  if (st != NOMAS_OK) return st;
+  if (n_parts < 1 || n_outs < 1)
+    return fail(NOMAS_ERR_INVALID_ARG, "need n_parts >= 1 and n_outs >= 1");
+  if (n_parts > NOMAS_MAX_MERGE_PARTS || n_outs > NOMAS_MAX_MERGE_OUTPUTS)
+    return fail(NOMAS_ERR_UNSUPPORTED, "at most %d parts and %d outputs (got %d, %d)",
+                NOMAS_MAX_MERGE_PARTS, NOMAS_MAX_MERGE_OUTPUTS, n_parts, n_outs);
+  if (n_q < 0 || n_q > 0x7fff0000LL || row0 < 0 || n_rows < 0 || row0 + n_rows > n_q)
+    return fail(NOMAS_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, n_q = %lld)",
+                (long long)row0, (long long)(row0 + n_rows), (long long)n_q);
+  if (n_rows == 0) return ok();
+  if (o_parts == nullptr || lse_parts == nullptr || o_outs == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "pointer tables missing");
+  const int64_t pb = n_q * kRowBytes, lb = n_q * kHeads * 4;
+  for (int r = 0; r < n_parts; ++r)
+    if (o_parts[r] == nullptr || lse_parts[r] == nullptr || !aligned16(o_parts[r]) ||
+        (reinterpret_cast<uintptr_t>(lse_parts[r]) & 3u))
+      return fail(NOMAS_ERR_INVALID_ARG, "part %d pointers missing or misaligned", r);
+  for (int k = 0; k < n_outs; ++k) {
+    float *lk = lse_outs != nullptr ? lse_outs[k] : nullptr;
+    if (o_outs[k] == nullptr || !aligned16(o_outs[k]) || (reinterpret_cast<uintptr_t>(lk) & 3u))
+      return fail(NOMAS_ERR_INVALID_ARG, "output %d pointers missing or misaligned", k);
+    for (int r = 0; r < n_parts; ++r)
+      if (overlap(o_outs[k], pb, o_parts[r], pb) || overlap(o_outs[k], pb, lse_parts[r], lb) ||
+          overlap(lk, lb, o_parts[r], pb) || overlap(lk, lb, lse_parts[r], lb))
+        return fail(NOMAS_ERR_INVALID_ARG, "output %d overlaps part %d", k, r);
+  }
+  const cudaError_t e = launch_merge_peers(
+      reinterpret_cast<const uint16_t *const *>(o_parts), lse_parts, n_parts, n_q, row0, n_rows,
+      reinterpret_cast<uint16_t *const *>(o_outs), lse_outs, n_outs,
+      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "peer merge launch");
+  return ok();
+}
+
 nomas_status nomas_segment_attention(const void *q, int64_t n_q, const nomas_kv_span *spans,
                                      int32_t n_spans, void *o, float *lse, float softmax_scale,
                                      int32_t heads, int32_t head_dim, int32_t *dev_err,

@@ -15,6 +15,14 @@
 // threads cover one 4 KiB row, so every part's row is one coalesced read),
 // four parts in flight at a time, and accumulates in fp32.
 // Traffic per row: R x (4 KiB + 64 B) read + 4 KiB + 64 B written.
+//
+// The same kernel serves two layouts of the partials: stacked in one buffer
+// (nomas_attention_merge, all rows, one output), or found through a table of
+// R pointers with a row range and up to 32 outputs (nomas_attention_merge_peers).
+// With pointers into other GPUs' memory, the table form is the exchange and
+// the merge in one kernel: each GPU reads the partial rows it owns from every
+// GPU and stores the merged rows into every GPU's output, with plain loads
+// and stores over NVLink.
 #include <cuda_bf16.h>
 
 #include "nomas_internal.h"
@@ -27,39 +35,72 @@ constexpr int kThreads = kRows * kHeads;   // phase 1: one (row, head) per threa
 constexpr int kWRow = kHeads + 1;          // padded [row][head] plane of one part
 constexpr int kWPlane = kRows * kWRow;
 
+// Where the R partial results live.  Stacked: one buffer, part r at a fixed
+// stride ([R][n_q][16][128] and [R][16][n_q]).  Table: R base pointers, any
+// of which may address another GPU's memory mapped into this process.
+struct StackedParts {
+  const uint16_t *o;
+  const float *lse;
+  int64_t n_q;
+  __device__ __forceinline__ const uint4 *o_row(int r, int64_t row) const {
+    return reinterpret_cast<const uint4 *>(o) + ((int64_t)r * n_q + row) * kRowVecs;
+  }
+  __device__ __forceinline__ float lse_at(int r, int h, int64_t row) const {
+    return lse[((int64_t)r * kHeads + h) * n_q + row];
+  }
+};
+struct TableParts {
+  const uint16_t *o[NOMAS_MAX_MERGE_PARTS];
+  const float *lse[NOMAS_MAX_MERGE_PARTS];
+  int64_t n_q;
+  __device__ __forceinline__ const uint4 *o_row(int r, int64_t row) const {
+    return reinterpret_cast<const uint4 *>(o[r]) + row * kRowVecs;
+  }
+  __device__ __forceinline__ float lse_at(int r, int h, int64_t row) const {
+    return lse[r][(int64_t)h * n_q + row];
+  }
+};
+// Where the merged rows go: every listed output gets the same rows ([n_q]
+// rows each; a null LSE pointer skips that output's LSE).
+struct Outputs {
+  uint16_t *o[NOMAS_MAX_MERGE_OUTPUTS];
+  float *lse[NOMAS_MAX_MERGE_OUTPUTS];
+  int32_t n;
+};
+
+template <class Parts>
 __global__ void __launch_bounds__(kThreads)
-merge_kernel(const uint16_t *__restrict__ o_parts, const float *__restrict__ lse_parts,
-             int32_t n_parts, int64_t n_q, uint16_t *__restrict__ o, float *__restrict__ lse) {
+merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
+             int64_t row_end, const Outputs outs) {
   extern __shared__ float w_s[];  // [n_parts][kRows][kWRow]
-  const int64_t row0 = (int64_t)blockIdx.x * kRows;
+  const int64_t row0 = row_begin + (int64_t)blockIdx.x * kRows;
   {
     const int h = threadIdx.x >> 4, rr = threadIdx.x & 15;
     const int64_t row = row0 + rr;
     float *w = w_s + rr * kWRow + h;
     float m = -INFINITY;
-    if (row < n_q)
-      for (int r = 0; r < n_parts; ++r)
-        m = fmaxf(m, lse_parts[((int64_t)r * kHeads + h) * n_q + row]);
+    if (row < row_end)
+      for (int r = 0; r < n_parts; ++r) m = fmaxf(m, parts.lse_at(r, h, row));
     float total = 0.f;
     for (int r = 0; r < n_parts; ++r) {
-      const float e =
-          m == -INFINITY ? 0.f : expf(lse_parts[((int64_t)r * kHeads + h) * n_q + row] - m);
+      const float e = m == -INFINITY ? 0.f : expf(parts.lse_at(r, h, row) - m);
       w[r * kWPlane] = e;
       total += e;
     }
     const float inv = total > 0.f ? 1.f / total : 0.f;
     for (int r = 0; r < n_parts; ++r) w[r * kWPlane] *= inv;
-    if (lse != nullptr && row < n_q)
-      lse[(int64_t)h * n_q + row] = total > 0.f ? m + logf(total) : -INFINITY;
+    if (row < row_end) {
+      const float l = total > 0.f ? m + logf(total) : -INFINITY;
+      for (int k = 0; k < outs.n; ++k)
+        if (outs.lse[k] != nullptr) outs.lse[k][(int64_t)h * n_q + row] = l;
+    }
   }
   __syncthreads();
   const int h = threadIdx.x >> 4, c = threadIdx.x & 15;
-  const int64_t part_vecs = n_q * kRowVecs;  // one part, in 16-byte chunks
   for (int i = 0; i < kRows; ++i) {
     const int64_t row = row0 + i;
-    if (row >= n_q) break;
+    if (row >= row_end) break;
     const float *w = w_s + i * kWRow + h;
-    const uint4 *src = reinterpret_cast<const uint4 *>(o_parts) + row * kRowVecs + h * 16 + c;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     auto add = [&](uint4 v, float wr) {
       const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
@@ -69,23 +110,25 @@ merge_kernel(const uint16_t *__restrict__ o_parts, const float *__restrict__ lse
         acc[2 * k + 1] = fmaf(wr, __uint_as_float(wd[k] & 0xffff0000u), acc[2 * k + 1]);
       }
     };
+    const int off = h * 16 + c;  // this thread's 16-byte chunk of the row
     int r = 0;
     for (; r + 4 <= n_parts; r += 4) {
       uint4 v[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = src[(int64_t)(r + k) * part_vecs];
+      for (int k = 0; k < 4; ++k) v[k] = parts.o_row(r + k, row)[off];
 #pragma unroll
       for (int k = 0; k < 4; ++k) add(v[k], w[(r + k) * kWPlane]);
     }
-    for (; r < n_parts; ++r) add(src[(int64_t)r * part_vecs], w[r * kWPlane]);
+    for (; r < n_parts; ++r) add(parts.o_row(r, row)[off], w[r * kWPlane]);
     uint32_t out[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
       out[k] = *reinterpret_cast<uint32_t *>(&b);
     }
-    reinterpret_cast<uint4 *>(o + row * kRowElems + h * kHeadDim)[c] =
-        make_uint4(out[0], out[1], out[2], out[3]);
+    const uint4 packed = make_uint4(out[0], out[1], out[2], out[3]);
+    for (int k = 0; k < outs.n; ++k)
+      reinterpret_cast<uint4 *>(outs.o[k] + row * kRowElems)[off] = packed;
   }
 }
 
@@ -97,8 +140,39 @@ cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_
   const int64_t blocks = (n_q + kRows - 1) / kRows;
   if (blocks > 0x7fffffff || n_parts > NOMAS_MAX_MERGE_PARTS) return cudaErrorInvalidValue;
   const size_t smem = (size_t)n_parts * kWPlane * sizeof(float);
-  merge_kernel<<<(unsigned)blocks, kThreads, smem, stream>>>(o_parts, lse_parts, n_parts, n_q, o,
-                                                              lse);
+  Outputs outs{};
+  outs.o[0] = o;
+  outs.lse[0] = lse;
+  outs.n = 1;
+  merge_kernel<StackedParts><<<(unsigned)blocks, kThreads, smem, stream>>>(
+      StackedParts{o_parts, lse_parts, n_q}, n_parts, n_q, 0, n_q, outs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_peers(const uint16_t *const *o_parts, const float *const *lse_parts,
+                               int32_t n_parts, int64_t n_q, int64_t row0, int64_t n_rows,
+                               uint16_t *const *o_outs, float *const *lse_outs, int32_t n_outs,
+                               cudaStream_t stream) {
+  if (n_rows <= 0) return cudaSuccess;
+  const int64_t blocks = (n_rows + kRows - 1) / kRows;
+  if (blocks > 0x7fffffff || n_parts < 1 || n_parts > NOMAS_MAX_MERGE_PARTS || n_outs < 1 ||
+      n_outs > NOMAS_MAX_MERGE_OUTPUTS)
+    return cudaErrorInvalidValue;
+  TableParts parts{};
+  for (int r = 0; r < n_parts; ++r) {
+    parts.o[r] = o_parts[r];
+    parts.lse[r] = lse_parts[r];
+  }
+  parts.n_q = n_q;
+  Outputs outs{};
+  for (int k = 0; k < n_outs; ++k) {
+    outs.o[k] = o_outs[k];
+    outs.lse[k] = lse_outs != nullptr ? lse_outs[k] : nullptr;
+  }
+  outs.n = n_outs;
+  const size_t smem = (size_t)n_parts * kWPlane * sizeof(float);
+  merge_kernel<TableParts><<<(unsigned)blocks, kThreads, smem, stream>>>(
+      parts, n_parts, n_q, row0, row0 + n_rows, outs);
   return cudaGetLastError();
 }
 

@@ -104,6 +104,12 @@ cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
 // ---------------------------------------------------------------- merge ----
 cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_t n_parts,
                          int64_t n_q, uint16_t *o, float *lse, cudaStream_t stream);
+// Rows [row0, row0 + n_rows) of n_parts partials found through pointer
+// tables (host arrays), written to n_outs outputs.
+cudaError_t launch_merge_peers(const uint16_t *const *o_parts, const float *const *lse_parts,
+                               int32_t n_parts, int64_t n_q, int64_t row0, int64_t n_rows,
+                               uint16_t *const *o_outs, float *const *lse_outs, int32_t n_outs,
+                               cudaStream_t stream);
 
 // ----------------------------------------------------------------- errors --
 // Sets the message nomas_last_error() returns on this thread; returns st.

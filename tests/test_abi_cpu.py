@@ -282,3 +282,28 @@ def test_split_attention_validation_and_scratch_size(lib):
         == nm.NOMAS_ERR_INVALID_ARG  # scratch overlaps a span
     assert f(FAKE, 100, spans, 1, o, lse, 0.0, 16, 64, 4, scr, need, None, None) \
         == nm.NOMAS_ERR_UNSUPPORTED
+
+
+def test_peer_merge_validation(lib):
+    P = ctypes.c_void_p
+
+    def table(*ptrs):
+        return (P * len(ptrs))(*ptrs)
+
+    parts, lses = table(FAKE, FAKE + 10 ** 9), table(FAKE + 2 * 10 ** 9, FAKE + 3 * 10 ** 9)
+    outs, louts = table(FAKE + 4 * 10 ** 9), table(FAKE + 5 * 10 ** 9)
+    f = lib.nomas_attention_merge_peers
+    assert f(parts, lses, 2, 100, 0, 0, outs, louts, 1, 16, 128, None) == nm.NOMAS_OK  # no rows
+    assert f(parts, lses, 0, 100, 0, 10, outs, louts, 1, 16, 128, None) == nm.NOMAS_ERR_INVALID_ARG
+    assert f(parts, lses, 2, 100, 0, 10, outs, louts, 0, 16, 128, None) == nm.NOMAS_ERR_INVALID_ARG
+    assert f(parts, lses, nm.MAX_MERGE_PARTS + 1, 100, 0, 10, outs, louts, 1, 16, 128, None) \
+        == nm.NOMAS_ERR_UNSUPPORTED
+    assert f(parts, lses, 2, 100, 0, 10, outs, louts, nm.MAX_MERGE_OUTPUTS + 1, 16, 128, None) \
+        == nm.NOMAS_ERR_UNSUPPORTED
+    assert f(parts, lses, 2, 100, 95, 10, outs, louts, 1, 16, 128, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # rows past n_q
+    assert f(parts, lses, 2, 100, 0, 10, outs, louts, 1, 16, 64, None) == nm.NOMAS_ERR_UNSUPPORTED
+    assert f(table(FAKE + 8, FAKE + 10 ** 9), lses, 2, 100, 0, 10, outs, louts, 1, 16, 128, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # misaligned part
+    assert f(parts, lses, 2, 100, 0, 10, table(FAKE + ROW), louts, 1, 16, 128, None) \
+        == nm.NOMAS_ERR_INVALID_ARG  # an output inside a part

@@ -58,3 +58,46 @@ def test_sharded_attention_single_rank_is_plain_attention():
     o2 = nm.segment_attention(q, spans)
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() <= 2 ** -7
+
+
+@pytest.mark.parametrize("world,n_q,n_k", [(3, 700, 4000), (2, 130, 300), (4, 1000, 2000)])
+def test_peer_merge_emulating_ranks_on_one_gpu(world, n_q, n_k):
+    # Each "GPU" is a set of buffers on this one: phase 1 runs for every rank,
+    # then phase 2 for every rank, in stream order (nothing waits on anything
+    # else).  Every rank's output must be the whole attention.
+    q, k, v = (randn_bf16((n, 16, 128), s) for n, s in ((n_q, 41), (n_k, 42), (n_k, 43)))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    part_o = [torch.empty((n_q, 16, 128), dtype=torch.bfloat16, device="cuda")
+              for _ in range(world)]
+    part_lse = [torch.empty((16, n_q), dtype=torch.float32, device="cuda") for _ in range(world)]
+    o_out = [torch.full((n_q, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+             for _ in range(world)]
+    lse_out = [torch.full((16, n_q), 7.0, dtype=torch.float32, device="cuda")
+               for _ in range(world)]
+    for r in range(world):
+        a, b = nm.shard_rows(n_k, r, world, align=128)
+        nm.peer_partial_attention(qd, [(kd[a:b], vd[a:b])], part_o[r], part_lse[r])
+    for r in range(world):
+        nm.peer_merge_owned_rows(part_o, part_lse, o_out, lse_out, r, world)
+    stacked = nm.attention_merge(torch.stack(part_o), torch.stack(part_lse))
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attention(f64(q), [(f64(k), f64(v))])
+    for r in range(world):
+        assert torch.equal(o_out[r].view(torch.int16), o_out[0].view(torch.int16))
+        assert torch.equal(lse_out[r], lse_out[0])
+    assert torch.equal(o_out[0].view(torch.int16), stacked.view(torch.int16))
+    assert_close(f64(o_out[0]), o_ref, what=f"peer merge over {world} ranks O")
+    assert_close(lse_out[0].cpu().double().numpy(), l_ref, what=f"peer merge over {world} ranks LSE")
+
+
+def test_peer_merge_writes_only_its_rows():
+    n_q = 300
+    parts = [randn_bf16((n_q, 16, 128), 50 + r).cuda() for r in range(2)]
+    lses = [torch.zeros((16, n_q), dtype=torch.float32, device="cuda") for _ in range(2)]
+    outs = [torch.full((n_q, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")]
+    nm.attention_merge_peers(parts, lses, outs, None, row0=100, n_rows=37)
+    torch.cuda.synchronize()
+    assert torch.all(outs[0][:100] == 7.0) and torch.all(outs[0][137:] == 7.0)
+    # equal LSEs: the merged rows are the average of the two parts, rounded once
+    want = (f64(parts[0][100:137]) + f64(parts[1][100:137])) / 2   # on the host, in fp64
+    assert_bf16_rounding(f64(outs[0][100:137]), want, what="average of two parts")
