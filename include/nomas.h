@@ -386,6 +386,37 @@ nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, 
                                    int32_t head_dim, void *stream);
 
 /*
+ * Key-sharded attention whose partial results go straight to their owners
+ * ("What 'world memory' stores": the cache spread over eight GPUs, sp_size 8;
+ * the routing is this library's design).  This GPU attends with every query
+ * row over its own key spans, as nomas_segment_attention does, but each query
+ * row's partial O and LSE are stored into part `slot` (this GPU's index) of
+ * the buffers of the GPU that owns the row, from the epilogue of the
+ * attention kernel, so the exchange runs while other tiles still compute.
+ * Each owner then merges its rows from its own buffers with
+ * nomas_attention_merge_peers (parts = its R slots, outputs = every GPU's O).
+ *   n_owners, owner_row0: owner s owns query rows [owner_row0[s],
+ *               owner_row0[s + 1]) (host int64[n_owners + 1], from 0 to n_q,
+ *               non-decreasing).
+ *   owner_o, owner_lse: host arrays of n_owners device pointers to each
+ *               owner's stacked buffers, [R][n_q][heads][head_dim] bf16 and
+ *               [R][heads][n_q] fp32, R > slot; only rows the owner owns are
+ *               written.  They may be other GPUs' memory mapped into this
+ *               process (peer access, CUDA IPC or symmetric memory).
+ *   slot      : 0 <= slot < NOMAS_MAX_MERGE_PARTS.
+ * The caller orders the owners' merges after every GPU's call (a cross-GPU
+ * barrier on the streams).  Other arguments as nomas_segment_attention.
+ * Errors: as nomas_segment_attention, plus NOMAS_ERR_INVALID_ARG for bad
+ * owner tables or buffers that overlap the inputs.
+ */
+nomas_status nomas_segment_attention_to_owners(const void *q, int64_t n_q,
+                                               const nomas_kv_span *spans, int32_t n_spans,
+                                               int32_t n_owners, const int64_t *owner_row0,
+                                               void *const *owner_o, float *const *owner_lse,
+                                               int32_t slot, float softmax_scale, int32_t heads,
+                                               int32_t head_dim, int32_t *dev_err, void *stream);
+
+/*
  * The merge of key-shard partials fused with their exchange between GPUs
  * ("What 'world memory' stores": the cache spread over eight GPUs, sp_size 8;
  * how the partial results meet is not on the page).  Each GPU calls it for

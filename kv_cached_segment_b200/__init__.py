@@ -63,6 +63,7 @@ EXPORTED_SYMBOLS = (
     "nomas_segment_attention_split",
     "nomas_segment_attention_scratch_bytes",
     "nomas_attention_merge_peers",
+    "nomas_segment_attention_to_owners",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -162,6 +163,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_segment_attention_scratch_bytes.argtypes = [I64, I32]
     lib.nomas_attention_merge_peers.restype = ctypes.c_int
     lib.nomas_attention_merge_peers.argtypes = [P, P, I32, I64, I64, I64, P, P, I32, I32, I32, P]
+    lib.nomas_segment_attention_to_owners.restype = ctypes.c_int
+    lib.nomas_segment_attention_to_owners.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, I32, P,
+                                                      P, P, I32, F32, I32, I32, P, P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -573,6 +577,61 @@ def peer_partial_attention(q, local_spans, part_o, part_lse):
     """Phase 1 of key-sharded attention over peer memory: this GPU's partial
     (O, LSE) over its own key spans, into its slot of the partial buffers."""
     segment_attention(q, local_spans, o=part_o, lse=part_lse.view(-1))
+
+
+def _span_table(spans):
+    arr = (_KVSpan * max(1, len(spans)))()
+    for i, (k, v) in enumerate(spans):
+        nk = _rows(k, f"span {i} k")
+        if _rows(v, f"span {i} v") != nk:
+            raise ValueError(f"span {i}: k and v differ in rows")
+        arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
+    return arr
+
+
+def owner_rows(n_q: int, world: int):
+    """Row boundaries of the owners: world + 1 ints, shares on 16-row steps."""
+    return [shard_rows(n_q, r, world, align=16)[0] for r in range(world)] + [n_q]
+
+
+def peer_attention_to_owners(q, local_spans, inbox_o_peers, inbox_lse_peers, slot: int,
+                             dev_err=None, stream=None):
+    """Phase 1 of key-sharded attention with the exchange in the attention
+    kernel: this GPU's partial (O, LSE) over its own key spans, each query
+    row stored into part ``slot`` of its owner's inbox (owner s owns the rows
+    of ``owner_rows(n_q, world)``, world = len(inbox_o_peers)).
+    inbox_o_peers[s]: bf16 [R][n_q][16][128]; inbox_lse_peers[s]: fp32
+    [R][16][n_q] (R > slot); they may live on other GPUs."""
+    lib = load_library()
+    n_q = _rows(q, "q")
+    world = len(inbox_o_peers)
+    if len(inbox_lse_peers) != world or world > MAX_MERGE_PARTS:
+        raise ValueError("one o and one lse inbox per owner, at most MAX_MERGE_PARTS owners")
+    for t in inbox_o_peers:
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape[0] <= slot or \
+                t.shape[1] != n_q or not t.is_contiguous():
+            raise ValueError("inbox_o_peers must be contiguous bf16 [R][n_q][16][128], R > slot")
+    for t in inbox_lse_peers:
+        if t.dtype != torch.float32 or t.dim() != 3 or t.shape[0] <= slot or \
+                t.shape[2] != n_q or not t.is_contiguous():
+            raise ValueError("inbox_lse_peers must be contiguous fp32 [R][16][n_q], R > slot")
+    rows = (ctypes.c_int64 * (world + 1))(*owner_rows(n_q, world))
+    o_tab = (ctypes.c_void_p * world)(*[t.data_ptr() for t in inbox_o_peers])
+    l_tab = (ctypes.c_void_p * world)(*[t.data_ptr() for t in inbox_lse_peers])
+    _check(lib.nomas_segment_attention_to_owners(_ptr(q), n_q, _span_table(local_spans),
+                                                 len(local_spans), world, rows, o_tab, l_tab,
+                                                 int(slot), 0.0, HEADS, HEAD_DIM, _ptr(dev_err),
+                                                 _stream(stream)))
+
+
+def peer_merge_inbox(inbox_o, inbox_lse, o_peers, lse_peers, rank: int, stream=None):
+    """Phase 2 with the exchange in the attention kernel: merge this GPU's own
+    rows from its inbox (local [R][n_q][16][128] and [R][16][n_q]) and store
+    them into every GPU's output."""
+    n_q = inbox_o.shape[1]
+    a, b = owner_rows(n_q, len(o_peers))[rank:rank + 2]
+    attention_merge_peers(list(inbox_o.unbind(0)), list(inbox_lse.unbind(0)), o_peers, lse_peers,
+                          row0=a, n_rows=b - a, stream=stream)
 
 
 def peer_merge_owned_rows(part_o_peers, part_lse_peers, o_peers, lse_peers, rank: int,

@@ -329,7 +329,15 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               float softmax_scale, int32_t heads, int32_t head_dim,
                               int32_t *dev_err, const nomas_attention_opts *opts,
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
-                              void *stream);
+                              const struct OwnerRouting *routing, void *stream);
+
+// Destination of owner-routed partial outputs (see AttnArgs::n_owners).
+struct OwnerRouting {
+  int32_t n_owners, slot;
+  const int64_t *row0;   // n_owners + 1 entries
+  void *const *o;        // n_owners stacked [R][n_q][16][128] buffers
+  float *const *lse;     // n_owners stacked [R][16][n_q] buffers
+};
 
 // Scratch of a key-split attention: S partial outputs [S][n_q][16][128] bf16,
 // then their LSEs [S][16][n_q] fp32.
@@ -520,7 +528,54 @@ nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_
                                         const nomas_attention_opts *opts, void *stream) {
   const ApiRange nvtx_range("nomas_segment_attention_ex");
   return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
-                          heads, head_dim, dev_err, opts, 1, nullptr, 0, stream);
+                          heads, head_dim, dev_err, opts, 1, nullptr, 0, nullptr, stream);
+}
+
+nomas_status nomas_segment_attention_to_owners(const void *q, int64_t n_q,
+                                               const nomas_kv_span *spans, int32_t n_spans,
+                                               int32_t n_owners, const int64_t *owner_row0,
+                                               void *const *owner_o, float *const *owner_lse,
+                                               int32_t slot, float softmax_scale, int32_t heads,
+                                               int32_t head_dim, int32_t *dev_err,
+                                               void *stream) {
+  const ApiRange nvtx_range("nomas_segment_attention_to_owners");
+  if (n_owners < 1 || n_owners > NOMAS_MAX_MERGE_PARTS)
+    return fail(NOMAS_ERR_INVALID_ARG, "n_owners must be in [1, %d] (got %d)",
+                NOMAS_MAX_MERGE_PARTS, n_owners);
+  if (slot < 0 || slot >= NOMAS_MAX_MERGE_PARTS)
+    return fail(NOMAS_ERR_INVALID_ARG, "slot must be in [0, %d) (got %d)", NOMAS_MAX_MERGE_PARTS,
+                slot);
+  if (owner_row0 == nullptr || owner_o == nullptr || owner_lse == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "owner tables are required");
+  if (owner_row0[0] != 0 || owner_row0[n_owners] != n_q)
+    return fail(NOMAS_ERR_INVALID_ARG, "owner rows must start at 0 and end at n_q");
+  const int64_t part_bytes = n_q * kRowBytes, part_lse = n_q * kHeads * 4;
+  for (int s = 0; s < n_owners; ++s) {
+    if (owner_row0[s + 1] < owner_row0[s])
+      return fail(NOMAS_ERR_INVALID_ARG, "owner rows must not decrease");
+    if (owner_o[s] == nullptr || owner_lse[s] == nullptr || !aligned16(owner_o[s]) ||
+        (reinterpret_cast<uintptr_t>(owner_lse[s]) & 3u))
+      return fail(NOMAS_ERR_INVALID_ARG, "owner %d buffers missing or misaligned", s);
+    // this rank's part of owner s's buffers must not overlap the inputs
+    const void *po = static_cast<const uint8_t *>(owner_o[s]) + (int64_t)slot * part_bytes;
+    const void *pl = reinterpret_cast<const uint8_t *>(owner_lse[s]) + (int64_t)slot * part_lse;
+    if (overlap(po, part_bytes, q, part_bytes) || overlap(pl, part_lse, q, part_bytes))
+      return fail(NOMAS_ERR_INVALID_ARG, "owner %d buffers overlap q", s);
+    for (int k = 0; k < n_spans && spans != nullptr; ++k) {
+      const int64_t sb = spans[k].len * kRowBytes;
+      if (overlap(po, part_bytes, spans[k].k, sb) || overlap(po, part_bytes, spans[k].v, sb) ||
+          overlap(pl, part_lse, spans[k].k, sb) || overlap(pl, part_lse, spans[k].v, sb))
+        return fail(NOMAS_ERR_INVALID_ARG, "owner %d buffers overlap span %d", s, k);
+    }
+  }
+  const OwnerRouting routing{n_owners, slot, owner_row0, owner_o, owner_lse};
+  // o and lse name this rank's part of the first owner's buffers: only their
+  // presence and alignment are checked; the kernel writes through the table.
+  void *o0 = static_cast<uint8_t *>(owner_o[0]) + (int64_t)slot * part_bytes;
+  float *l0 = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(owner_lse[0]) +
+                                        (int64_t)slot * part_lse);
+  return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o0, l0, softmax_scale,
+                          heads, head_dim, dev_err, nullptr, 1, nullptr, 0, &routing, stream);
 }
 
 int64_t nomas_segment_attention_scratch_bytes(int64_t n_q, int32_t kv_splits) {
@@ -537,7 +592,7 @@ nomas_status nomas_segment_attention_split(const void *q, int64_t n_q, const nom
   const ApiRange nvtx_range("nomas_segment_attention_split");
   return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
                           heads, head_dim, dev_err, nullptr, kv_splits, scratch, scratch_bytes,
-                          stream);
+                          nullptr, stream);
 }
 
 nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
@@ -556,7 +611,7 @@ nomas_status nomas_segment_attention_sparse(const void *q, int64_t n_q,
     return fail(NOMAS_ERR_INVALID_ARG, "tile_list and tile_count must be 4-byte aligned");
   return attention_common(q, n_q, spans, n_spans, tile_list, tile_count, max_tiles, o, lse,
                           softmax_scale, heads, head_dim, dev_err, nullptr, 1, nullptr, 0,
-                          stream);
+                          nullptr, stream);
 }
 
 }  // extern "C"
@@ -569,7 +624,7 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               float softmax_scale, int32_t heads, int32_t head_dim,
                               int32_t *dev_err, const nomas_attention_opts *opts,
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
-                              void *stream) {
+                              const OwnerRouting *routing, void *stream) {
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   if (kv_splits < 1 || kv_splits > NOMAS_MAX_MERGE_PARTS)
@@ -626,6 +681,17 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   a.tile_count = tile_count;
   a.max_tiles = max_tiles;
   if (n_used == 0) {
+    if (routing != nullptr) {
+      // no keys: O = 0, LSE = -inf in this rank's part of every owner's buffers
+      for (int s = 0; s < routing->n_owners; ++s) {
+        const cudaError_t e = launch_attention_empty(
+            static_cast<uint16_t *>(routing->o[s]) + (int64_t)routing->slot * n_q * kRowElems,
+            routing->lse[s] + (int64_t)routing->slot * kHeads * n_q, n_q,
+            static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "attention (no keys) launch");
+      }
+      return ok();
+    }
     const cudaError_t e = launch_attention_empty(static_cast<uint16_t *>(o), lse, n_q,
                                                  static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention (no keys) launch");
@@ -639,6 +705,16 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   a.o = static_cast<uint16_t *>(o);
   a.lse = lse;
   a.kv_splits = 1;
+  a.n_owners = 0;
+  if (routing != nullptr) {
+    a.n_owners = routing->n_owners;
+    a.owner_slot = routing->slot;
+    for (int s = 0; s <= routing->n_owners; ++s) a.owner_row0[s] = routing->row0[s];
+    for (int s = 0; s < routing->n_owners; ++s) {
+      a.owner_o[s] = static_cast<uint16_t *>(routing->o[s]);
+      a.owner_lse[s] = routing->lse[s];
+    }
+  }
   uint16_t *part_o = nullptr;
   float *part_lse = nullptr;
   if (kv_splits > 1) {

@@ -719,10 +719,22 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       }
     }
     // Epilogue: O / l -> bf16, LSE = ln(2) * (m + log2 l), into part
-    // blockIdx.z of the outputs when the keys are split.
-    uint16_t *const o_out = p.o + (int64_t)blockIdx.z * p.n_q * kRowElems;
-    float *const lse_out =
-        p.lse == nullptr ? nullptr : p.lse + (int64_t)blockIdx.z * kHeads * p.n_q;
+    // blockIdx.z of the outputs when the keys are split, or into part
+    // owner_slot of the buffers of the row's owner when the outputs are
+    // routed (those may be other GPUs' memory: plain stores over NVLink).
+    const int64_t my_row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
+    uint16_t *o_base = p.o;
+    float *lse_base = p.lse;
+    int64_t part = blockIdx.z;
+    if (p.n_owners > 0) {
+      int s = 0;
+      while (s + 1 < p.n_owners && my_row >= p.owner_row0[s + 1]) ++s;
+      o_base = p.owner_o[s];
+      lse_base = p.owner_lse[s];
+      part = p.owner_slot;
+    }
+    uint16_t *const o_out = o_base + part * p.n_q * kRowElems;
+    float *const lse_out = lse_base == nullptr ? nullptr : lse_base + part * kHeads * p.n_q;
     bool have_o = ok && n_kv > 0;
     if (have_o) have_o = __all_sync(0xffffffffu, wait_phase(bar(kBarOFull + tile), 0, ctl));
     if (have_o) {

@@ -96,6 +96,16 @@ struct AttnArgs {
   // writes its partial O and LSE to part z of o ([S][n_q][16][128]) and lse
   // ([S][16][n_q]).  1: no split.
   int32_t kv_splits;
+  // Owner-routed partial outputs (key-sharded attention over peer memory):
+  // when n_owners > 0, query row i belongs to the owner s with
+  // owner_row0[s] <= i < owner_row0[s + 1], and its O and LSE go to part
+  // owner_slot of that owner's stacked buffers owner_o[s] ([R][n_q][16][128])
+  // and owner_lse[s] ([R][16][n_q]) instead of o and lse.
+  int32_t n_owners;
+  int32_t owner_slot;
+  int64_t owner_row0[NOMAS_MAX_MERGE_PARTS + 1];
+  uint16_t *owner_o[NOMAS_MAX_MERGE_PARTS];
+  float *owner_lse[NOMAS_MAX_MERGE_PARTS];
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,

@@ -307,3 +307,27 @@ def test_peer_merge_validation(lib):
         == nm.NOMAS_ERR_INVALID_ARG  # misaligned part
     assert f(parts, lses, 2, 100, 0, 10, table(FAKE + ROW), louts, 1, 16, 128, None) \
         == nm.NOMAS_ERR_INVALID_ARG  # an output inside a part
+
+
+def test_routed_attention_validation(lib):
+    P = ctypes.c_void_p
+    spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, 500))
+    o_tab = (P * 2)(FAKE + 3 * 10 ** 9, FAKE + 4 * 10 ** 9)
+    l_tab = (P * 2)(FAKE + 5 * 10 ** 9, FAKE + 6 * 10 ** 9)
+    f = lib.nomas_segment_attention_to_owners
+
+    def rows(*r):
+        return (ctypes.c_int64 * len(r))(*r)
+
+    def call(n_owners=2, row0=rows(0, 64, 100), o=o_tab, lse=l_tab, slot=1, q=FAKE):
+        return f(q, 100, spans, 1, n_owners, row0, o, lse, slot, 0.0, 16, 128, None, None)
+
+    assert call(n_owners=0) == nm.NOMAS_ERR_INVALID_ARG
+    assert call(n_owners=nm.MAX_MERGE_PARTS + 1) == nm.NOMAS_ERR_INVALID_ARG
+    assert call(slot=nm.MAX_MERGE_PARTS) == nm.NOMAS_ERR_INVALID_ARG
+    assert call(row0=rows(1, 64, 100)) == nm.NOMAS_ERR_INVALID_ARG      # must start at 0
+    assert call(row0=rows(0, 64, 99)) == nm.NOMAS_ERR_INVALID_ARG       # must end at n_q
+    assert call(row0=rows(0, 80, 60)) == nm.NOMAS_ERR_INVALID_ARG      # must end at n_q
+    assert call(n_owners=3, row0=rows(0, 80, 60, 100)) == nm.NOMAS_ERR_INVALID_ARG  # decreasing
+    assert call(o=(P * 2)(FAKE + 3 * 10 ** 9 + 8, FAKE + 4 * 10 ** 9)) == nm.NOMAS_ERR_INVALID_ARG
+    assert call(q=FAKE + 3 * 10 ** 9 + 100 * ROW) == nm.NOMAS_ERR_INVALID_ARG  # q in a part

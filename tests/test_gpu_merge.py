@@ -101,3 +101,44 @@ def test_peer_merge_writes_only_its_rows():
     # equal LSEs: the merged rows are the average of the two parts, rounded once
     want = (f64(parts[0][100:137]) + f64(parts[1][100:137])) / 2   # on the host, in fp64
     assert_bf16_rounding(f64(outs[0][100:137]), want, what="average of two parts")
+
+
+@pytest.mark.parametrize("world,n_q,n_k", [(3, 700, 4000), (4, 130, 300), (2, 1000, 2000)])
+def test_attention_routed_to_owners_emulating_ranks_on_one_gpu(world, n_q, n_k):
+    # Phase 1 on every "GPU": its partial rows go straight into part `rank`
+    # of each row owner's inbox; phase 2 on every "GPU": the owner merges its
+    # rows from its inbox into every output.  With n_k = 300 over 4 ranks,
+    # rank 0 has no keys and stores O = 0, LSE = -inf.
+    q, k, v = (randn_bf16((n, 16, 128), s) for n, s in ((n_q, 61), (n_k, 62), (n_k, 63)))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    inbox_o = [torch.full((world, n_q, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+               for _ in range(world)]
+    inbox_l = [torch.full((world, 16, n_q), 7.0, dtype=torch.float32, device="cuda")
+               for _ in range(world)]
+    o_out = [torch.full((n_q, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+             for _ in range(world)]
+    lse_out = [torch.full((16, n_q), 7.0, dtype=torch.float32, device="cuda")
+               for _ in range(world)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for r in range(world):
+        a, b = nm.shard_rows(n_k, r, world, align=128)
+        nm.peer_attention_to_owners(qd, [(kd[a:b], vd[a:b])], inbox_o, inbox_l, slot=r,
+                                    dev_err=err)
+    for r in range(world):
+        nm.peer_merge_inbox(inbox_o[r], inbox_l[r], o_out, lse_out, r)
+    # the same partials computed the plain way, merged by the stacked kernel
+    parts_o, parts_l = [], []
+    for r in range(world):
+        a, b = nm.shard_rows(n_k, r, world, align=128)
+        l_r = torch.empty(16 * n_q, dtype=torch.float32, device="cuda")
+        parts_o.append(nm.segment_attention(qd, [(kd[a:b], vd[a:b])], lse=l_r))
+        parts_l.append(l_r.view(16, n_q))
+    stacked = nm.attention_merge(torch.stack(parts_o), torch.stack(parts_l))
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for r in range(world):
+        assert torch.equal(o_out[r].view(torch.int16), stacked.view(torch.int16))
+        assert torch.equal(lse_out[r], lse_out[0])
+    o_ref, l_ref = oracle.attention(f64(q), [(f64(k), f64(v))])
+    assert_close(f64(o_out[0]), o_ref, what=f"routed attention over {world} ranks O")
+    assert_close(lse_out[0].cpu().double().numpy(), l_ref, what=f"routed over {world} ranks LSE")
