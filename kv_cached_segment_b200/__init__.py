@@ -634,6 +634,23 @@ def peer_merge_inbox(inbox_o, inbox_lse, o_peers, lse_peers, rank: int, stream=N
                           row0=a, n_rows=b - a, stream=stream)
 
 
+def sharded_segment_attention_routed(q, local_spans, inbox_o_peers, inbox_lse_peers, o_peers,
+                                     lse_peers, rank: int, barrier=lambda: None, dev_err=None):
+    """Key-sharded attention with the exchange in the attention kernel, on
+    the GPU of ``rank``: phase 1 (partials stored into the owners' inboxes),
+    ``barrier()``, phase 2 (this GPU's rows merged into every output),
+    ``barrier()``.  The lists hold every GPU's buffers, mapped into this
+    process (peer access, IPC or symmetric memory); ``barrier`` must order
+    the streams of all GPUs (a one-element NCCL all-reduce, for example).
+    Returns this GPU's output, o_peers[rank]."""
+    peer_attention_to_owners(q, local_spans, inbox_o_peers, inbox_lse_peers, slot=rank,
+                             dev_err=dev_err)
+    barrier()
+    peer_merge_inbox(inbox_o_peers[rank], inbox_lse_peers[rank], o_peers, lse_peers, rank)
+    barrier()
+    return o_peers[rank]
+
+
 def peer_merge_owned_rows(part_o_peers, part_lse_peers, o_peers, lse_peers, rank: int,
                           world: int):
     """Phase 2: this GPU merges the query rows it owns (a contiguous share,

@@ -142,3 +142,19 @@ def test_attention_routed_to_owners_emulating_ranks_on_one_gpu(world, n_q, n_k):
     o_ref, l_ref = oracle.attention(f64(q), [(f64(k), f64(v))])
     assert_close(f64(o_out[0]), o_ref, what=f"routed attention over {world} ranks O")
     assert_close(lse_out[0].cpu().double().numpy(), l_ref, what=f"routed over {world} ranks LSE")
+
+
+def test_routed_sharded_attention_on_one_rank_is_plain_attention():
+    q = randn_bf16((300, 16, 128), 71).cuda()
+    k, v = randn_bf16((900, 16, 128), 72).cuda(), randn_bf16((900, 16, 128), 73).cuda()
+    inbox_o = [torch.empty((1, 300, 16, 128), dtype=torch.bfloat16, device="cuda")]
+    inbox_l = [torch.empty((1, 16, 300), dtype=torch.float32, device="cuda")]
+    o_out = [torch.empty((300, 16, 128), dtype=torch.bfloat16, device="cuda")]
+    l_out = [torch.empty((16, 300), dtype=torch.float32, device="cuda")]
+    o = nm.sharded_segment_attention_routed(q, [(k, v)], inbox_o, inbox_l, o_out, l_out, rank=0)
+    lse = torch.empty(16 * 300, dtype=torch.float32, device="cuda")
+    plain = nm.segment_attention(q, [(k, v)], lse=lse)
+    torch.cuda.synchronize()
+    # one part with weight 1: the merge only re-rounds values already in bf16
+    assert torch.equal(o.view(torch.int16), plain.view(torch.int16))
+    assert torch.allclose(l_out[0].view(-1), lse, atol=1e-5)
