@@ -18,9 +18,16 @@ Entry points (same names as the C ABI, without the ``nomas_`` prefix):
 - ``temporal_context_frames``: the power-spaced history frame picker (host).
 
 Holders: ``KVCache`` and ``KVCacheI8`` (caller-owned device buffers plus
-``len``), ``RopeConfig`` and ``SegLayout``.  ``sharded_segment_attention``
-runs key-sharded attention over the ranks of a ``torch.distributed`` group
-(partial attention per rank, all-gather of the partials, merge).
+``len``), ``RopeConfig`` and ``SegLayout``.
+
+Key-sharded attention over several GPUs, in three forms:
+``sharded_segment_attention`` (partial attention per rank, NCCL all-gather of
+the partials, merge); ``peer_partial_attention`` + ``peer_merge_owned_rows``
+(the all-gather replaced by a merge that reads the owned rows of every GPU's
+partial over peer memory and writes every GPU's output,
+``attention_merge_peers``); and ``sharded_segment_attention_routed``
+(``peer_attention_to_owners`` stores the partial rows into their owners'
+buffers from the attention kernel itself, then ``peer_merge_inbox``).
 """
 from __future__ import annotations
 
