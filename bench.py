@@ -455,6 +455,20 @@ def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
     return flops / elapsed / 1e12, done, elapsed, blas_threads(), parity
 
 
+def cpu_model() -> str:
+    """The host CPU's model name and logical core count."""
+    name = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{name}, {os.cpu_count()} logical cores"
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -602,7 +616,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(step, LayerStep):
         rate, rows, secs, threads, parity = cpu_oracle_rate(step, budget_s=12.0,
                                                             rows_per_chunk=16, max_rows=512)
-        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "host": cpu_model(),
                "sample": f"fp64 oracle RoPE + attention of {rows} sampled segment query rows "
                          f"x 16 heads over all {step.w.n_k} keys ({secs:.1f} s)"}
         if step.sparse is not None:
@@ -790,6 +804,7 @@ def run_reference(args, rank, world):
                    "l2": "host memory (the oracle runs on the CPU)",
                    "parallelism": "one process on the host cores"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "host": cpu_model(),
                          "sample": f"fp64 oracle RoPE + attention of {rows_per_step} sampled "
                                    f"segment query rows per step x 16 heads over all {w.n_k} "
                                    f"keys, {args.steps} steps"},
