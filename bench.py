@@ -659,7 +659,7 @@ def main():
                      "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 {peak_kind}",
                      "traffic": recorded_traffic(args.workload)},
         "cpu_baseline": cpu, "e2e": e2e, "parity": parity,
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": step.launches_per_step * args.steps * world,  # all ranks
         "clocks": clocks,
     }
     if n_shards:
