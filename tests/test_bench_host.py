@@ -85,3 +85,14 @@ def test_sparse_tile_lists_pad_with_minus_one():
     lists, counts = sparse_tile_lists(100, [300], keep_spans=[], candidate_spans=[0],
                                       fraction=0.0, seed=1)
     assert (counts == 0).all() and (lists == -1).all() and lists.shape[-1] == 1
+
+
+def test_owner_rows_partition_the_queries_on_16_row_steps():
+    for n_q, world in ((28112, 8), (700, 3), (130, 4), (15, 2), (0, 3)):
+        rows = nm.owner_rows(n_q, world)
+        assert len(rows) == world + 1 and rows[0] == 0 and rows[-1] == n_q
+        assert all(a <= b for a, b in zip(rows, rows[1:]))
+        assert all(r % 16 == 0 for r in rows[:-1])
+        # the same shares as the merge of owned rows uses
+        for r in range(world):
+            assert (rows[r], rows[r + 1]) == nm.shard_rows(n_q, r, world, align=16)
