@@ -93,3 +93,49 @@ def test_sparse_deterministic():
     o1, l1, _ = _run(q, spans, lists, counts)
     o2, l2, _ = _run(q, spans, lists, counts)
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
+@pytest.mark.slow
+def test_sparse_720p_layer_step_sampled_blocks():
+    # The bench's block-sparse configuration at full size: the 720p
+    # layer-step (RoPE + append on the GPU), every text tile and a seeded 25%
+    # of the history and segment tiles per 256-query block and head.  Three
+    # query blocks are checked against the oracle, each as its own one-block
+    # problem (its 256 rows with its own tile lists).
+    from seeded_inputs import WORKLOADS, layer_inputs
+
+    w = WORKLOADS["720p"]
+    inp = layer_inputs(w, seed=5)
+    ns = w.n_seg
+    lay = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, w.n_text)
+    cache = nm.KVCache.empty(w.n_cache + ns, w.tokens_per_frame)
+    cache.k[:w.n_cache] = inp["cache_k"].cuda()
+    cache.v[:w.n_cache] = inp["cache_v"].cuda()
+    cache.len = w.n_cache
+    q, k, v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
+    q_rot = torch.empty_like(q)
+    nm.kvcache_append(cache, k[:ns], v[:ns], q_in=q, q_out=q_rot, layout=lay, cfg=nm.RopeConfig())
+    lens = [w.n_cache, w.n_text, ns]
+    lists, counts = sparse_tile_lists(w.n_q, lens, keep_spans=[1], candidate_spans=[0, 2],
+                                      fraction=0.25, seed=5)
+    spans = [cache.span(0, w.n_cache), (k[ns:], v[ns:]), cache.span(w.n_cache, w.n_cache + ns)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lse = torch.empty(16 * w.n_q, dtype=torch.float32, device="cuda")
+    o = nm.segment_attention_sparse(q_rot, spans, torch.from_numpy(lists).cuda(),
+                                    torch.from_numpy(counts).cuda(), lse=lse, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+
+    t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    qf = oracle.rope3d(f64(inp["q"]), ns, t, h, ww)
+    kf = oracle.rope3d(f64(inp["k"][:ns]), ns, t, h, ww)
+    spans_f = [(f64(inp["cache_k"]), f64(inp["cache_v"])),
+               (f64(inp["k"][ns:]), f64(inp["v"][ns:])), (kf, f64(inp["v"][:ns]))]
+    lse_g = lse.view(16, -1).cpu().numpy().astype(np.float64)
+    last = lists.shape[0] - 1
+    for b in (0, 57, last):      # first, middle (video rows) and last (text rows) blocks
+        rows = np.arange(b * 256, min(w.n_q, (b + 1) * 256))
+        tl = [[lists[b, hh, :counts[b, hh]].tolist() for hh in range(16)]]
+        o_ref, l_ref = oracle.block_sparse_attention(qf[rows], spans_f, tl)
+        assert_close(f64(o[torch.as_tensor(rows)]), o_ref, what=f"720p sparse block {b} O")
+        assert_close(lse_g[:, rows], l_ref, what=f"720p sparse block {b} LSE")
