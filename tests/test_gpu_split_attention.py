@@ -68,3 +68,38 @@ def test_split_with_no_keys():
     empty = torch.empty((0, 16, 128), dtype=torch.bfloat16)
     o, lse = _run(q, [(empty, empty)], 4)
     assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+@pytest.mark.slow
+def test_short_layer_step_with_automatic_splits_sampled_rows():
+    # The bench's short configuration (3.35 waves of query blocks, so the
+    # automatic choice splits the keys), sampled rows against the oracle.
+    from seeded_inputs import WORKLOADS, layer_inputs
+
+    w = WORKLOADS["short"]
+    inp = layer_inputs(w, seed=6)
+    ns = w.n_seg
+    lay = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, w.n_text)
+    cache = nm.KVCache.empty(w.n_cache + ns, w.tokens_per_frame)
+    cache.k[:w.n_cache] = inp["cache_k"].cuda()
+    cache.v[:w.n_cache] = inp["cache_v"].cuda()
+    cache.len = w.n_cache
+    q, k, v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
+    q_rot = torch.empty_like(q)
+    nm.kvcache_append(cache, k[:ns], v[:ns], q_in=q, q_out=q_rot, layout=lay, cfg=nm.RopeConfig())
+    spans = [cache.span(0, w.n_cache), (k[ns:], v[ns:]), cache.span(w.n_cache, w.n_cache + ns)]
+    assert nm.auto_kv_splits(w.n_q, [w.n_cache, w.n_text, ns]) > 1
+    lse = torch.empty(16 * w.n_q, dtype=torch.float32, device="cuda")
+    o = nm.segment_attention(q_rot, spans, lse=lse, kv_splits="auto")
+    torch.cuda.synchronize()
+    t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    qf = oracle.rope3d(f64(inp["q"]), ns, t, h, ww)
+    kf = oracle.rope3d(f64(inp["k"][:ns]), ns, t, h, ww)
+    rows = np.unique(np.concatenate([np.random.default_rng(2).integers(0, w.n_q, 40),
+                                     [0, ns - 1, ns, w.n_q - 1]]))
+    o_ref, l_ref = oracle.attention_rows(
+        qf, rows, [(f64(inp["cache_k"]), f64(inp["cache_v"])),
+                   (f64(inp["k"][ns:]), f64(inp["v"][ns:])), (kf, f64(inp["v"][:ns]))])
+    assert_close(f64(o[torch.as_tensor(rows)]), o_ref, what="short, split keys, O")
+    got_l = lse.view(16, -1)[:, torch.as_tensor(rows).cuda()].cpu().numpy().astype(np.float64)
+    assert_close(got_l, l_ref, what="short, split keys, LSE")
