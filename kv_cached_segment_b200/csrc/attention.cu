@@ -40,6 +40,8 @@
 // Every wait is bounded (a globaltimer limit); on expiry the kernel records
 // NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and
 // returns.
+#include <atomic>
+
 #include <cuda_bf16.h>
 
 #include "nomas_internal.h"
@@ -798,20 +800,22 @@ __global__ void attention_empty_kernel(uint16_t *o, float *lse, int64_t n_q) {
 }  // namespace
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
-  // The shared-memory opt-in is a per-device function attribute.
-  static bool attr_set[64] = {};
+  // The shared-memory opt-in is a per-device function attribute.  Several
+  // host threads may make their first call on a device at once: the
+  // attribute calls are idempotent, and the flag is atomic.
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(attention_kernel<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemAlloc);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t q_blocks = ((int64_t)a.n_q + kQTiles * kBM - 1) / (kQTiles * kBM);
   if (q_blocks <= 0) return cudaSuccess;
