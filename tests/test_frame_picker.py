@@ -3,7 +3,6 @@ import ctypes
 import json
 import os
 
-import numpy as np
 import pytest
 
 import kv_cached_segment_b200 as nm

@@ -8,7 +8,7 @@ import torch
 import kv_cached_segment_b200 as nm
 import oracle
 from seeded_inputs import WORKLOADS, bounded_frame_list, layer_inputs, randn_bf16
-from tests._util import assert_close, bits, f64
+from tests._util import assert_close, f64
 
 pytestmark = pytest.mark.gpu
 

@@ -5,7 +5,7 @@ import torch
 
 import kv_cached_segment_b200 as nm
 import oracle
-from seeded_inputs import WORKLOADS, bounded_frame_list, random_frame_list, randn_bf16
+from seeded_inputs import WORKLOADS, random_frame_list, randn_bf16
 from tests._util import assert_close, bits, f64
 
 pytestmark = pytest.mark.gpu

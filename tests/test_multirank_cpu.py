@@ -7,7 +7,6 @@ world of two processes.
 import os
 import socket
 
-import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

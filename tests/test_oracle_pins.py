@@ -14,7 +14,6 @@ import os
 import numpy as np
 import pytest
 
-import oracle
 from oracle import nomas_oracle as O
 
 COS1 = 0.5403023058681398   # cos(1 rad)
