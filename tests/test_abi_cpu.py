@@ -331,3 +331,31 @@ def test_routed_attention_validation(lib):
     assert call(n_owners=3, row0=rows(0, 80, 60, 100)) == nm.NOMAS_ERR_INVALID_ARG  # decreasing
     assert call(o=(P * 2)(FAKE + 3 * 10 ** 9 + 8, FAKE + 4 * 10 ** 9)) == nm.NOMAS_ERR_INVALID_ARG
     assert call(q=FAKE + 3 * 10 ** 9 + 100 * ROW) == nm.NOMAS_ERR_INVALID_ARG  # q in a part
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    # The boundary is a C ABI: the header must compile as C99 with no
+    # warnings, and a C program must link against the library and call it.
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler on this machine")
+    src = tmp_path / "use_nomas.c"
+    src.write_text(
+        '#include "nomas.h"\n'
+        '#include <stdio.h>\n'
+        'int main(void) {\n'
+        '  int32_t frames[18], n = 0;\n'
+        '  nomas_status st = nomas_temporal_context_frames(360, 18, 2.0f, frames, 18, &n);\n'
+        '  printf("%d %d %d %s\\n", (int)st, (int)n, (int)frames[0], nomas_version());\n'
+        '  return st == NOMAS_OK ? 0 : 1;\n'
+        '}\n')
+    exe = tmp_path / "use_nomas"
+    lib_dir = os.path.dirname(nm.library_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lnomas",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0] == "0" and int(out[1]) > 0 and out[2] == "0"
