@@ -215,7 +215,9 @@ typedef struct {
 } nomas_kvcache_i8;
 
 /*
- * nomas_kvcache_append into an INT8 cache: the rotated segment keys (rounded
+ * nomas_kvcache_append into an INT8 cache ("The 4090 preset": the finished
+ * segment's K/V are quantised to one byte per value once, when they are
+ * written to the cache): the rotated segment keys (rounded
  * to bf16, as the bf16 path would store them) and the values are quantised
  * per (token, head): a = absmax, stored scale = a / 127, code =
  * rint(x * (127 / a)), divisions and product rounded to nearest in fp32 and
@@ -229,7 +231,9 @@ nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
                                      const nomas_rope3d_cfg *cfg, void *stream);
 
 /*
- * nomas_kvcache_select from an INT8 cache into a bf16 window: the listed
+ * nomas_kvcache_select from an INT8 cache into a bf16 window ("The 4090
+ * preset": the chosen past frames are restored to the GPU before each
+ * segment): the listed
  * frames are restored to the GPU-side window as bf16(fp32(code * scale))
  * (product rounded to nearest in fp32, then to bf16 nearest-even).  Same
  * arguments, index checks and errors as nomas_kvcache_select.
@@ -270,8 +274,9 @@ typedef struct {
 } nomas_attention_opts;
 
 /*
- * nomas_segment_attention with per-call options (opts may be NULL for the
- * defaults); identical otherwise.
+ * nomas_segment_attention ("How one segment is made": the joint attention of
+ * the segment and the text over the history and themselves) with per-call
+ * options (opts may be NULL for the defaults); identical otherwise.
  */
 nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_kv_span *spans,
                                         int32_t n_spans, void *o, float *lse, float softmax_scale,

@@ -359,3 +359,17 @@ def test_header_is_plain_c_and_links_from_c(tmp_path):
                     f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert out[0] == "0" and int(out[1]) > 0 and out[2] == "0"
+
+
+def test_every_entry_point_cites_its_passage():
+    # Each call's comment names the section of the pages that defines the
+    # operation (a quoted title), or says that the pages have no counterpart.
+    text = open(os.path.join(ROOT, "include", "nomas.h")).read()
+    for m in re.finditer(r"nomas_status\s+(nomas_[a-z0-9_]+)\s*\(", text):
+        before = text[:m.start()]
+        end = before.rfind("*/")
+        start = before.rfind("/*", 0, end)
+        between = [ln for ln in before[end + 2:].splitlines() if ln.strip()]
+        assert all(ln.startswith("#define") for ln in between), m.group(1)
+        comment = before[start:end]
+        assert '"' in comment or "no counterpart" in comment, m.group(1)
