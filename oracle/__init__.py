@@ -24,6 +24,8 @@ from .nomas_oracle import (  # noqa: F401
     f32_to_bf16_bits,
     quantize_int8,
     dequantize_int8,
+    dequantize_int8_f64,
+    round_to_bf16_bits,
     key_tiles,
     block_sparse_attention,
     merge_partials,

@@ -239,29 +239,55 @@ def quantize_int8(x_bits):
     [KV] "The 4090 preset": the cache is quantised once per segment to one
     byte per value plus an FP32 scale per token and head (4,224 B per token
     per layer for K and V together).  Reading (the page gives no formula):
-    absmax scaling decided in float32: a = max_d |x_d|, scale = a / 127 (the
-    stored scale) and code = rint(x_d * (127 / a)), each division and the
-    product rounded to nearest in float32 and rint rounding half to even; an
-    all-zero (token, head) gets scale 0 and codes 0.
-    Returns int8 codes [N][H][D] and float32 scales [N][H].
+    absmax scaling, a = max_d |x_d|; the stored scale is a / 127 rounded to
+    the nearest float32, and the code is the integer nearest to the exact
+    quotient 127 x_d / a, ties to even.  An all-zero (token, head) gets scale
+    0 and codes 0.  Returns int8 codes [N][H][D] and float32 scales [N][H].
+
+    The quotient is formed in float64 from the exactly widened inputs: 127 x
+    is exact, and the one rounding of the division cannot move a quotient
+    onto or across a half-integer (x and a carry 8 significant bits, so a
+    quotient that is not itself a tie stays more than 2^-17 away from one).
     """
-    x = bf16_bits_to_f64(x_bits).astype(np.float32)          # exact
+    x = bf16_bits_to_f64(x_bits)                               # exact
     amax = np.max(np.abs(x), axis=2)                           # exact
-    scale = (amax / np.float32(127.0)).astype(np.float32)      # fp32 RN
+    scale = (amax.astype(np.float32) / np.float32(127.0)).astype(np.float32)
     zero = amax == 0
-    safe = np.where(zero, np.float32(1.0), amax).astype(np.float32)
-    inv = (np.float32(127.0) / safe).astype(np.float32)        # fp32 RN
-    q = (x * inv[:, :, None]).astype(np.float32)               # fp32 RN
-    codes = np.clip(np.rint(q), -127, 127).astype(np.int8)
+    safe = np.where(zero, 1.0, amax)
+    codes = np.rint(127.0 * x / safe[:, :, None])              # half to even
+    codes = np.clip(codes, -127, 127).astype(np.int8)          # |x| <= a
     codes[zero] = 0
     return codes, scale
 
 
+def round_to_bf16_bits(x) -> np.ndarray:
+    """Round float64 values to the nearest bf16, ties to even, in one step; bits.
+
+    bf16 keeps 8 significant bits: a normal value in [2^e, 2^(e+1)) lies on
+    the grid of step 2^(e-7), and below 2^-126 the step is 2^-133 (the bf16
+    subnormals).  The value is divided by its step (exact: a power of two),
+    rounded to an integer half to even, and multiplied back.  Inputs are
+    finite and inside the bf16 range.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                       # |x| in [2^(e-1), 2^e)
+    step_exp = np.maximum(e - 1 - 7, -133)
+    step = np.ldexp(1.0, step_exp)
+    r = np.rint(x / step) * step             # exact in float64
+    return f32_to_bf16_bits(r.astype(np.float32))   # r is a bf16 value: exact
+
+
+def dequantize_int8_f64(codes, scales) -> np.ndarray:
+    """Dequantised values code * scale, exact in float64 ([KV] "The 4090
+    preset": a stored value is its code times its token and head's scale)."""
+    return (np.asarray(codes, dtype=np.float64) *
+            np.asarray(scales, dtype=np.float32).astype(np.float64)[:, :, None])
+
+
 def dequantize_int8(codes, scales) -> np.ndarray:
-    """bf16 bits of code * scale (product in float32, then rounded to bf16)."""
-    prod = (np.asarray(codes, dtype=np.float32) *
-            np.asarray(scales, dtype=np.float32)[:, :, None]).astype(np.float32)
-    return f32_to_bf16_bits(prod)
+    """bf16 bits of code * scale: the exact product rounded once to the
+    nearest bf16, ties to even (the restored window is bf16)."""
+    return round_to_bf16_bits(dequantize_int8_f64(codes, scales))
 
 
 # ---------------------------------------------------------------------------

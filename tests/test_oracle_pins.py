@@ -400,6 +400,98 @@ def test_int8_error_bound_and_exact_grid():
     assert np.array_equal(O.dequantize_int8(c2, s2), g)
 
 
+def test_int8_hand_ties_round_half_to_even():
+    # Row 0: a = 127, so the code is the nearest integer to x itself: 0.5 -> 0,
+    # 1.5 -> 2, 2.5 -> 2, -2.5 -> -2, 126.5 -> 126 (ties to even), 3.25 -> 3,
+    # -127 -> -127.  Row 1: a = 2, x = a / 2 gives 63.5 -> 64 and x = -a
+    # gives -127.  Every x is a bf16 value.
+    x = np.zeros((2, 1, 128))
+    x[0, 0, :8] = [127.0, 0.5, 1.5, 2.5, -2.5, 126.5, 3.25, -127.0]
+    x[1, 0, :3] = [1.0, -2.0, -1.0]
+    codes, scales = O.quantize_int8(_bits_of(x))
+    assert codes[0, 0, :8].tolist() == [127, 0, 2, 2, -2, 126, 3, -127]
+    assert codes[1, 0, :3].tolist() == [64, -127, -64]
+    assert np.all(codes[:, :, 8:] == 0)
+    assert scales[0, 0] == np.float32(1.0) and scales[1, 0] == np.float32(2.0 / 127.0)
+
+
+def test_int8_codes_equal_exact_rational_rounding():
+    # Brute force with exact rationals: Python's round() of a Fraction rounds
+    # half to even with no floating point at all.
+    from fractions import Fraction
+
+    r = rng(22)
+    x = _bits_of(r.standard_normal((6, 3, 128)) * np.array([1e-3, 1.0, 40.0])[None, :, None])
+    codes, scales = O.quantize_int8(x)
+    xf = O.bf16_bits_to_f64(x)
+    for t in range(x.shape[0]):
+        for h in range(x.shape[1]):
+            a = max(Fraction(float(v)) for v in np.abs(xf[t, h]))
+            for d in range(128):
+                want = round(127 * Fraction(float(xf[t, h, d])) / a)
+                assert codes[t, h, d] == want
+
+
+def test_int8_near_ties_the_fp32_reciprocal_route_misses():
+    # A quotient formed as x * fl(127 / a) in float32 can land on the wrong
+    # side of a half-integer; the plain definition must not.  Count that such
+    # inputs occur in this sample, then check every code exactly.
+    from fractions import Fraction
+
+    r = rng(23)
+    x = _bits_of(r.standard_normal((400, 16, 128)))
+    codes, _ = O.quantize_int8(x)
+    xf = O.bf16_bits_to_f64(x)
+    a = np.max(np.abs(xf), axis=2)
+    inv = (np.float32(127.0) / a.astype(np.float32)).astype(np.float32)
+    fp32_route = np.rint((xf.astype(np.float32) * inv[:, :, None]).astype(np.float32))
+    diff = np.argwhere(fp32_route != codes)
+    assert len(diff) > 0
+    for t, h, d in diff:
+        want = round(127 * Fraction(float(xf[t, h, d])) / Fraction(float(a[t, h])))
+        assert codes[t, h, d] == want
+
+
+def test_round_to_bf16_single_rounding():
+    # Ties between neighbours go to the even pattern; a value just above a tie
+    # goes up, just below goes down; subnormal steps are 2^-133.
+    t = 1.0 + 2.0 ** -8
+    vals = [t, t + 2.0 ** -40, t - 2.0 ** -40, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0,
+            3 * 2.0 ** -134, 2.0 ** -135]
+    got = O.round_to_bf16_bits(np.array(vals)).tolist()
+    assert got == [0x3F80, 0x3F81, 0x3F80, 0x3F82, 0xC020, 0x0000, 0x0002, 0x0000]
+
+
+def test_dequantize_rounds_the_exact_product_once():
+    # These (code, scale) pairs were found by search: their float32 product
+    # lands exactly on a bf16 tie although the exact product does not, so
+    # rounding to float32 first and then to bf16 can pick the wrong
+    # neighbour.  The oracle must equal exact rational rounding.
+    from fractions import Fraction
+
+    pairs = [(-60, 1026381141), (-67, 1028386999), (127, 998607638), (86, 1025239088),
+             (-101, 1026275591)]
+    got = []
+    for c, sb in pairs:
+        s = np.array([[np.uint32(sb)]], dtype=np.uint32).view(np.float32)
+        one = np.zeros((1, 1, 128), dtype=np.int8)
+        one[0, 0, 0] = c
+        got.append(int(O.dequantize_int8(one, s)[0, 0, 0]))
+    twice = 0
+    for (c, sb), g in zip(pairs, got):
+        s = float(np.uint32(sb).view(np.float32))
+        p = Fraction(c) * Fraction(s)
+        # exact nearest bf16 by brute force over the two float32-grid neighbours
+        lo_bits = O.f32_to_bf16_bits(np.float32(float(p)))  # a candidate
+        cands = {int(lo_bits) + k for k in (-1, 0, 1)}
+        best = min(cands, key=lambda b: (abs(Fraction(float(O.bf16_bits_to_f64(
+            np.array([b], dtype=np.uint16))[0])) - p), b & 1))
+        assert g == best
+        double = int(O.f32_to_bf16_bits(np.float32(c) * np.float32(s)))
+        twice += double != best
+    assert twice > 0  # the sample does separate the two roundings
+
+
 def test_int8_zero_rows():
     z = np.zeros((2, 3, 128), dtype=np.uint16)
     codes, scales = O.quantize_int8(z)
