@@ -47,11 +47,10 @@ __device__ __forceinline__ uint4 rot_chunk(uint4 v, const float (&c)[4], const f
   return v;
 }
 
-// Symmetric INT8 quantisation per (token, head): stored scale = a / 127 and
-// code = rint(x * (127 / a)) with a = max |x| over the head's 128 values; the
-// two divisions and the product round to nearest in float32 and rint rounds
-// half to even, so the codes are reproducible bit for bit; an all-zero head
-// gets scale 0 and codes 0.
+// Symmetric INT8 quantisation per (token, head): with a = max |x| over the
+// head's 128 values, the stored scale is a / 127 rounded to float32 and the
+// code is the integer nearest to the exact quotient 127 x / a, ties to even;
+// an all-zero head gets scale 0 and codes 0.
 //
 // A thread holds 8 values of each of 4 items (the keys, or the values, of 4
 // heads) of its row.  The absmax of the 4 items over the row's 16 lanes is a
@@ -91,23 +90,42 @@ __device__ __forceinline__ float row_absmax_transposed(const float (&am)[kHeadGr
   return fmaxf(r, __shfl_xor_sync(row_mask, r, 1));
 }
 
-// 8 codes of one chunk.  |x * inv| <= 127 (1 + 2^-24)^2 < 127.5, so adding
-// 1.5 * 2^23 rounds the product to an integer half to even and leaves it,
-// in two's complement, in the low byte of the sum; no clamp is needed.  The
-// product must be rounded to float32 before the add (a fused multiply-add
-// would round x * (127 / a) = 63.5 - tiny, common when x = a / 2, down to
-// 63 instead of 63.5 -> 64; a version written with the packed f32x2
-// multiply and add gave exactly those codes), so both steps use the scalar
-// intrinsics that are never contracted.
-__device__ __forceinline__ uint2 quant_chunk(uint4 v, float inv) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+// 8 codes of one chunk.  Fast path: p = x * inv with inv = 127 / a, both
+// rounded to float32, is within 127 * 2^-23 < 2^-15 of the exact quotient
+// 127 x / a; adding 1.5 * 2^23 rounds p to an integer half to even and leaves
+// it, in two's complement, in the low byte of the sum (|p| < 127.5, so no
+// clamp is needed).  That integer is the exact quotient's nearest unless p
+// lies within 2^-15 of a half-integer.  There the value takes the exact path:
+// 127 x is exact in float32 and the correctly rounded quotient
+// fl(127 x / a) cannot sit on a half-integer unless the exact quotient does
+// (x and a carry 8 significant bits, so a quotient that is not a tie is more
+// than 2^-17 from one, above half a float32 step below 128), so rounding it
+// half to even gives the code (also used when a is so small that 127 / a
+// overflows).  The product is rounded to float32 before the
+// add: the scalar intrinsics below are never contracted into a fused
+// multiply-add.
+__device__ __forceinline__ uint32_t round_magic(float x) {
+  return __float_as_uint(__fadd_rn(x, 12582912.0f));  // 1.5 * 2^23
+}
+__device__ __forceinline__ uint2 quant_chunk(uint4 v, float inv, float amax) {
+  constexpr float kMagic = 12582912.0f;
+  constexpr float kNearTie = 0.5f - 1.0f / 32768.0f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t t[8];
+  float x[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    t[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w[i] << 16), inv), kMagic));
-    t[2 * i + 1] =
-        __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w[i] & 0xffff0000u), inv), kMagic));
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+  uint32_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float p = __fmul_rn(x[i], inv);
+    t[i] = round_magic(p);
+    const float r = __fsub_rn(__uint_as_float(t[i]), kMagic);  // exact
+    // near a tie (exact difference), or 127 / a overflowed (a below ~3.7e-37)
+    if (fabsf(__fsub_rn(p, r)) >= kNearTie || !(fabsf(p) < 128.f))
+      t[i] = round_magic(__fdiv_rn(__fmul_rn(x[i], 127.f), amax));
   }
   const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040),
                                   0x5410);
@@ -212,8 +230,10 @@ rope_append_kernel(const __grid_constant__ RopeArgs a) {
         for (int g = 0; g < kHeadGroup; ++g) {
           // 8 codes per thread at [row][head][8cc..8cc+7]
           const int64_t coff = row * (kRowElems / 8) + (int64_t)(h0 + g) * 16 + cc;
-          const float inv_g = __shfl_sync(row_mask, inv, (threadIdx.x & 16) + 4 * g);
-          reinterpret_cast<uint2 *>(codes)[coff] = quant_chunk(src[g], inv_g);
+          const int owner = (threadIdx.x & 16) + 4 * g;
+          const float inv_g = __shfl_sync(row_mask, inv, owner);
+          const float amax_g = __shfl_sync(row_mask, amax, owner);
+          reinterpret_cast<uint2 *>(codes)[coff] = quant_chunk(src[g], inv_g, amax_g);
         }
       };
       if (do_k) {

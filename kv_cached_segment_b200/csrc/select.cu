@@ -56,11 +56,25 @@ select_kernel(const __grid_constant__ SelectArgs a, const __grid_constant__ Sele
 }
 
 // Gather + dequantize: window rows of frame j receive code * scale of source
-// frame idx[j], the product rounded to fp32 then to bf16 (nearest-even).  A
+// frame idx[j], the exact product rounded once to the nearest bf16 (ties to
+// even).  A
 // thread handles 8 codes (one 16-byte bf16 output chunk) per step: 4,224 B
 // read (codes + scales, K and V) and 8 KiB written per selected token.
 constexpr int kDqUnroll = 4;
 constexpr int kDqTile = kThreads * kDqUnroll;  // chunks of 8 codes per block
+
+// code * scale rounded to float32 "to odd": truncated toward zero, with the
+// last bit set when the truncation dropped anything.  The product of a 7-bit
+// code and a 24-bit scale has at most 31 significant bits, so the fused
+// multiply-add residual below is exact and is zero exactly when the product
+// is.  bf16 keeps 8 significant bits, at least two fewer than float32's 24,
+// so rounding the round-to-odd float32 to the nearest bf16 gives the nearest
+// bf16 of the exact product: no double-rounding error.
+__device__ __forceinline__ float product_round_to_odd(float code, float scale) {
+  const float r = __fmul_rz(code, scale);
+  const float e = __fmaf_rn(code, scale, -r);
+  return __uint_as_float(__float_as_uint(r) | (e != 0.f ? 1u : 0u));
+}
 
 __global__ void __launch_bounds__(kThreads)
 select_i8_kernel(const __grid_constant__ SelectI8Args a, const __grid_constant__ SelectHostList hl) {
@@ -105,7 +119,8 @@ select_i8_kernel(const __grid_constant__ SelectI8Args a, const __grid_constant__
       for (int i = 0; i < 4; ++i) {
         const float lo = (float)(int8_t)((w[i / 2] >> (16 * (i & 1))) & 0xff);
         const float hi = (float)(int8_t)((w[i / 2] >> (16 * (i & 1) + 8)) & 0xff);
-        __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(lo, sv[u]), __fmul_rn(hi, sv[u]));
+        __nv_bfloat162 b = __floats2bfloat162_rn(product_round_to_odd(lo, sv[u]),
+                                                 product_round_to_odd(hi, sv[u]));
         o[i] = *reinterpret_cast<uint32_t *>(&b);
       }
       dst[dst_row0 * kRowVecs + c] = make_uint4(o[0], o[1], o[2], o[3]);

@@ -27,10 +27,43 @@ def test_append_plain_quantisation_is_bit_exact():
     nm.kvcache_append_i8(cache, k.to(torch.bfloat16).cuda(), v.cuda())
     torch.cuda.synchronize()
     assert cache.len == 7 + n
+    near_ties = 0
     for codes, scales, src in ((cache.k, cache.k_scale, k), (cache.v, cache.v_scale, v)):
         want_c, want_s = oracle.quantize_int8(bits(src.to(torch.bfloat16)))
         assert np.array_equal(_codes(codes[7:7 + n]), want_c)
         assert np.array_equal(scales[7:7 + n].cpu().numpy().view(np.uint32), want_s.view(np.uint32))
+        near_ties += _fp32_reciprocal_route_misses(src, want_c)
+    # the sample holds quotients near half-integers, where x * fl(127 / a)
+    # in float32 alone would give the wrong code
+    print(f"codes the float32 reciprocal route would miss: {near_ties}")
+    assert near_ties > 0
+
+
+def _fp32_reciprocal_route_misses(src, want_codes):
+    x = f64(src.to(torch.bfloat16)).astype(np.float32)
+    a = np.max(np.abs(x), axis=2)
+    inv = (np.float32(127.0) / np.where(a == 0, np.float32(1), a)).astype(np.float32)
+    route = np.rint((x * inv[:, :, None]).astype(np.float32))
+    return int(np.count_nonzero(route != want_codes))
+
+
+def test_append_hand_ties():
+    # a = 127 per head: codes are x rounded half to even; a = 2: a / 2 -> 64.
+    x = torch.zeros((3, 16, 128))
+    x[0, :, :8] = torch.tensor([127.0, 0.5, 1.5, 2.5, -2.5, 126.5, 3.25, -127.0])
+    x[1, :, :3] = torch.tensor([1.0, -2.0, -1.0])
+    x[2, :, 0] = 2.0 ** -130  # absmax so small that 127 / a overflows float32
+    xb = x.to(torch.bfloat16)
+    cache = nm.KVCacheI8.empty(3, 1)
+    nm.kvcache_append_i8(cache, xb.cuda(), xb.cuda())
+    torch.cuda.synchronize()
+    got = _codes(cache.k)
+    assert got[0, :, :8].tolist() == [[127, 0, 2, 2, -2, 126, 3, -127]] * 16
+    assert got[1, :, :3].tolist() == [[64, -127, -64]] * 16
+    assert np.all(got[2, :, 0] == 127) and np.all(got[2, :, 1:] == 0)
+    want_c, want_s = oracle.quantize_int8(bits(xb))
+    assert np.array_equal(got, want_c) and np.array_equal(_codes(cache.v), want_c)
+    assert np.array_equal(cache.k_scale.cpu().numpy().view(np.uint32), want_s.view(np.uint32))
 
 
 def test_append_rotated_keys_within_quantisation_error():
@@ -83,6 +116,28 @@ def test_select_dequantises_bit_exactly(n_src, tpf, n_sel):
         want = oracle.dequantize_int8(oracle.kvcache_select(codes, idx, tpf),
                                       oracle.kvcache_select(scales, idx, tpf))
         assert np.array_equal(bits(dev), want)
+
+
+def test_select_dequantises_with_one_rounding():
+    # Random float32 scales make some float32 products land on a bf16 tie that
+    # the exact product is not on; rounding twice (float32, then bf16) would
+    # pick the wrong neighbour there.  The gather must equal the one-step
+    # rounding of the oracle everywhere, those cases included.
+    kk, vv, src = _i8_source(16, 920, 7)
+    idx = np.arange(16)[::-1].copy()
+    win = nm.KVCache.empty(16 * 920, 0)
+    nm.kvcache_select(src, idx.tolist(), win)
+    torch.cuda.synchronize()
+    twice = 0
+    for dev, (codes, scales) in ((win.k, kk), (win.v, vv)):
+        c = oracle.kvcache_select(codes, idx, 920)
+        s = oracle.kvcache_select(scales, idx, 920)
+        want = oracle.dequantize_int8(c, s)
+        assert np.array_equal(bits(dev), want)
+        prod32 = (c.astype(np.float32) * s[:, :, None]).astype(np.float32)
+        twice += int(np.count_nonzero(oracle.f32_to_bf16_bits(prod32) != want))
+    print(f"elements where rounding twice would differ: {twice}")
+    assert twice > 0
 
 
 def test_select_int8_device_list_bad_index():
