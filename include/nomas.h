@@ -219,10 +219,10 @@ typedef struct {
  * segment's K/V are quantised to one byte per value once, when they are
  * written to the cache): the rotated segment keys (rounded
  * to bf16, as the bf16 path would store them) and the values are quantised
- * per (token, head): a = absmax, stored scale = a / 127, code =
- * rint(x * (127 / a)), divisions and product rounded to nearest in fp32 and
- * rint rounding half to even; an all-zero (token, head) gets scale 0 and
- * codes 0.  Q is handled exactly as
+ * per (token, head): with a = absmax, the stored scale is a / 127 rounded to
+ * the nearest fp32, and the code is the integer nearest to the exact
+ * quotient 127 x / a, ties to even; an all-zero (token, head) gets scale 0
+ * and codes 0.  Q is handled exactly as
  * in nomas_kvcache_append.  Same errors as nomas_kvcache_append.
  */
 nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
@@ -234,13 +234,37 @@ nomas_status nomas_kvcache_append_i8(nomas_kvcache_i8 *cache, const void *k_seg,
  * nomas_kvcache_select from an INT8 cache into a bf16 window ("The 4090
  * preset": the chosen past frames are restored to the GPU before each
  * segment): the listed
- * frames are restored to the GPU-side window as bf16(fp32(code * scale))
- * (product rounded to nearest in fp32, then to bf16 nearest-even).  Same
+ * frames are restored to the GPU-side window as bf16 values: the exact
+ * product code * scale rounded once to the nearest bf16, ties to even.  Same
  * arguments, index checks and errors as nomas_kvcache_select.
  */
 nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
                                      int32_t n_frames, int32_t idx_on_device,
                                      nomas_kvcache *window, int32_t *dev_err, void *stream);
+
+/*
+ * nomas_kvcache_select from an INT8 cache into an INT8 window ("The 4090
+ * preset": the chosen past frames are kept on the GPU in INT8, 4,224 B per
+ * token per layer): the listed frames' codes and scales are copied bit for
+ * bit, nothing is dequantised; the window is then read by
+ * nomas_segment_attention_i8.  Window rows [j*P, (j+1)*P) of k, v, k_scale
+ * and v_scale receive source rows [idx[j]*P, (idx[j]+1)*P).  The window
+ * needs capacity >= n_frames * P; its tokens_per_frame is set to P and, on
+ * success, its len to n_frames * P.  Same frame lists, index checks and
+ * errors as nomas_kvcache_select.
+ */
+nomas_status nomas_kvcache_select_i8_codes(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
+                                           int32_t n_frames, int32_t idx_on_device,
+                                           nomas_kvcache_i8 *window, int32_t *dev_err,
+                                           void *stream);
+
+/* A contiguous run of `len` rows of an INT8 cache: codes [len][heads][head_dim]
+ * int8 and scales [len][heads] fp32, for K and V; value = code * scale. */
+typedef struct {
+  const void *k, *v;
+  const float *k_scale, *v_scale;
+  int64_t len;
+} nomas_kv_span_i8;
 
 /*
  * Power-spaced choice of the past latent frames to keep resident ("The 4090
@@ -261,8 +285,9 @@ nomas_status nomas_temporal_context_frames(int32_t n_past, int32_t budget, float
  *   wait_limit_ns: time limit of every pipeline wait inside the kernel
  *                  (0 selects the default of 2 s).  A wait that runs out sets
  *                  NOMAS_DEVERR_WAIT_TIMEOUT in *dev_err; the affected query
- *                  block then writes no output, releases its resources and
- *                  exits, and the CUDA context stays usable.
+ *                  block then sets its rows of O (and LSE) to NaN, releases
+ *                  its resources and exits, and the CUDA context stays
+ *                  usable.  The same holds in every attention entry point.
  *   testing_skip_kv_load: -1 in normal use.  For tests of the timeout path
  *                  only: a value k >= 0 makes every block leave out its k-th
  *                  K/V tile load (loads alternate K, V, K, V ... over the key
@@ -281,6 +306,34 @@ typedef struct {
 nomas_status nomas_segment_attention_ex(const void *q, int64_t n_q, const nomas_kv_span *spans,
                                         int32_t n_spans, void *o, float *lse, float softmax_scale,
                                         int32_t heads, int32_t head_dim, int32_t *dev_err,
+                                        const nomas_attention_opts *opts, void *stream);
+
+/*
+ * nomas_segment_attention over a history held in INT8 ("The 4090 preset":
+ * the resident past frames stay on the GPU in INT8; "Hy-Nomas en una RTX
+ * 4090", section "El preset de una GPU": stored in INT8, computed in BF16).
+ * The keys are `history` (dequantised: value = code * scale) followed by the
+ * bf16 `spans` (e.g. text, segment); every query row attends to all of them
+ * with no mask, exactly as nomas_segment_attention over the dequantised
+ * history.  The kernel converts each 128-key tile of codes to bf16
+ * (code * scale rounded to fp32, then to bf16 nearest-even) in shared
+ * memory on its way to the tensor cores; the history is never expanded in
+ * device memory.
+ *   history : host struct; its len may be 0 (then this is
+ *             nomas_segment_attention over `spans`).  Codes 16-byte
+ *             aligned, scales 16-byte aligned.
+ *   spans   : host array of n_spans bf16 runs, 1 + n_spans <=
+ *             NOMAS_MAX_SPANS.
+ *   opts    : as nomas_segment_attention_ex (may be NULL).
+ * Other arguments and errors as nomas_segment_attention_ex; a build whose
+ * INT8 kernel did not compile to the register allocation it assumes returns
+ * NOMAS_ERR_CUDA before launching anything.
+ */
+nomas_status nomas_segment_attention_i8(const void *q, int64_t n_q,
+                                        const nomas_kv_span_i8 *history,
+                                        const nomas_kv_span *spans, int32_t n_spans, void *o,
+                                        float *lse, float softmax_scale, int32_t heads,
+                                        int32_t head_dim, int32_t *dev_err,
                                         const nomas_attention_opts *opts, void *stream);
 
 /*
@@ -356,15 +409,20 @@ int64_t nomas_segment_attention_scratch_bytes(int64_t n_q, int32_t kv_splits);
  *   NOMAS_ERR_CAPACITY with a message giving both sizes, before anything is
  *   launched.
  *   The array is held on every device that uses this call until the process
- *   exits.  The first call on a device looks up the array's device address
- *   (with that device current) and keeps it: make that first call before any
- *   stream capture begins.
+ *   exits.  Its device address is looked up (with the device current) on
+ *   every call made outside stream capture and kept per device; a call made
+ *   while its stream is capturing uses the kept address.  So make one call
+ *   on a device before any stream capture begins, and one after a reset of
+ *   the device's primary context (cudaDeviceReset), which moves the array.
  *   Every call shares the array: calls that can run at the same time on the
  *   GPU (different streams, or different host threads) race on it and must
  *   be ordered by the caller.  Each call writes every byte of scratch it
- *   reads, so a call never sees the previous call's contents.
+ *   reads (a block whose pipeline wait ran out writes NaN rows, and its
+ *   output rows come out NaN), so a call never sees the previous call's
+ *   contents.
  * Errors: as nomas_segment_attention_split, plus NOMAS_ERR_CAPACITY (the
- * request exceeds the array) and NOMAS_ERR_CUDA (the address lookup failed).
+ * request exceeds the array) and NOMAS_ERR_CUDA (the address lookup failed,
+ * or no address is known yet and the stream is capturing).
  */
 nomas_status nomas_segment_attention_split_noalloc(const void *q, int64_t n_q,
                                                    const nomas_kv_span *spans, int32_t n_spans,
@@ -382,7 +440,9 @@ nomas_status nomas_segment_attention_split_noalloc(const void *q, int64_t n_q,
  *   lse_parts: [n_parts][heads][n_q] fp32 partial LSEs (natural log, device).
  *   o        : [n_q][heads][head_dim] bf16 output; lse: optional [heads][n_q].
  * Parts with LSE = -inf are empty and contribute nothing; if all are empty the
- * row gets O = 0 and LSE = -inf.  Outputs must not overlap the inputs.
+ * row gets O = 0 and LSE = -inf.  A part with a NaN LSE (a partial whose
+ * attention block ran out of time) makes the row's O and LSE NaN.  Outputs
+ * must not overlap the inputs.
  * 1 <= n_parts <= NOMAS_MAX_MERGE_PARTS (more returns NOMAS_ERR_UNSUPPORTED).
  * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.
  */

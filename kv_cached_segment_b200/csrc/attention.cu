@@ -38,8 +38,8 @@
 // exceed 2^16.
 //
 // Every wait is bounded (a globaltimer limit); on expiry the kernel records
-// NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, frees TMEM and
-// returns.
+// NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, sets the
+// block's rows of O and LSE to NaN, frees TMEM and returns.
 #include <atomic>
 
 #include <cuda_bf16.h>
@@ -57,32 +57,56 @@ constexpr int kQTiles = 2;
 #ifndef NOMAS_ATTN_STAGES
 #define NOMAS_ATTN_STAGES 5
 #endif
-constexpr int kStages = NOMAS_ATTN_STAGES;  // K/V ring slots
 constexpr uint32_t kTileBytes = kBN * kHeadDim * 2;   // 32 KiB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;       // 64 dims x 128 rows
+constexpr uint32_t kCodeTileBytes = kBN * kHeadDim;   // 16 KiB of INT8 codes
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kConvWarp0 = 12;        // INT8 variant: warps 12-15 dequantise
 constexpr uint32_t kTmemCols = 512;
 
-// Shared-memory map (offsets from a 1024-B aligned base).
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kOffQ + kQTiles * kTileBytes;
-constexpr uint32_t kOffBar = kOffKV + kStages * kTileBytes;
-// barrier indices (8 B each)
-constexpr int kBarQFull = 0;
-constexpr int kBarKVFull = 1;                      // + slot
-constexpr int kBarKVEmpty = kBarKVFull + kStages;  // + slot
-constexpr int kBarSFull = kBarKVEmpty + kStages;   // + tile
-constexpr int kBarPFull = kBarSFull + 2;           // + tile
-constexpr int kBarPHalf = kBarPFull + 2;           // + tile: first 64 keys of P
-constexpr int kBarOFull = kBarPHalf + 2;           // + tile
-constexpr int kBarDrain = kBarOFull + 2;
-constexpr int kNumBars = kBarDrain + 1;
-constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
-constexpr uint32_t kSmemUsed = kOffAbort + 4;
-constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base
+// Shared-memory map (offsets from a 1024-B aligned base) and thread count of
+// the two variants: bf16 spans only (10 warps, 5 ring slots), or a first span
+// held as INT8 codes + scales (16 warps: a converter warpgroup is added; 4
+// ring slots, 2 staging slots for code tiles).
+template <bool kI8>
+struct Cfg {
+  static constexpr int kStages = kI8 ? 4 : NOMAS_ATTN_STAGES;  // K/V ring slots
+  static constexpr int kThreads = kI8 ? 512 : 320;
+  static constexpr int kStaging = kI8 ? 2 : 0;
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = kOffQ + kQTiles * kTileBytes;
+  static constexpr uint32_t kOffStage = kOffKV + kStages * kTileBytes;
+  static constexpr uint32_t kOffBar = kOffStage + kStaging * kCodeTileBytes;
+  // barrier indices (8 B each)
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarKVFull = 1;                      // + slot
+  static constexpr int kBarKVEmpty = kBarKVFull + kStages;  // + slot
+  static constexpr int kBarSFull = kBarKVEmpty + kStages;   // + tile
+  static constexpr int kBarPFull = kBarSFull + 2;           // + tile
+  static constexpr int kBarPHalf = kBarPFull + 2;           // + tile: first 64 keys of P
+  static constexpr int kBarOFull = kBarPHalf + 2;           // + tile
+  static constexpr int kBarDrain = kBarOFull + 2;
+  static constexpr int kBarStFull = kBarDrain + 1;          // + staging slot
+  static constexpr int kBarStEmpty = kBarStFull + kStaging; // + staging slot
+  static constexpr int kNumBars = kBarStEmpty + kStaging;
+  static constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+  static constexpr uint32_t kSmemUsed = kOffAbort + 4;
+  static constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base
+};
+static_assert(Cfg<true>::kSmemAlloc <= 232448 && Cfg<false>::kSmemAlloc <= 232448,
+              "shared memory per block");
+
+// Register split of the INT8 variant (setmaxnreg, per warpgroup): the block
+// is launched with 512 threads x 128 registers = 65,536; the two softmax
+// warpgroups raise theirs to 168 and the producer/MMA and converter
+// warpgroups lower theirs to 88: 2 x 128 x 168 + 2 x 128 x 88 = 65,536.
+constexpr int kI8LaunchRegs = 128;
+constexpr int kI8SoftmaxRegs = 168;
+constexpr int kI8OtherRegs = 88;
+static_assert(2 * 128 * kI8SoftmaxRegs + 2 * 128 * kI8OtherRegs <= 512 * kI8LaunchRegs,
+              "register split exceeds the block's launch allocation");
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D,
 // M = 128, N = 128; A K-major; B K-major (QK^T: K rows are key-major with
@@ -324,7 +348,74 @@ __device__ __forceinline__ void issue_pv_half(uint32_t d_tmem, uint32_t p_tmem, 
            (k > 0) ? 1u : accumulate);
 }
 
-__device__ __forceinline__ int num_tiles(int64_t len) { return (int)((len + kBN - 1) / kBN); }
+// ------------------------------------------------- INT8 tile dequantisation --
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t (&w)[4]) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t *w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3])
+               : "memory");
+}
+// Makes this thread's shared-memory stores visible to the tensor core (the
+// async proxy), before the barrier that hands the tile over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// The converter warpgroup's own named barrier (id 1, 128 threads); the
+// reduction form returns the AND of every thread's flag, so that all of them
+// take the same branch after a bounded wait.
+__device__ __forceinline__ bool converters_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void converters_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Dequantises one key row of an INT8 code tile into a bf16 ring slot:
+// 128 codes become bf16(code * scale) (product rounded to float32, then to
+// bf16 nearest-even), written in the layout TMA gives a bf16 tile: two
+// 64-dim halves of 128 rows x 128 B, the 16-byte chunk j of row r at
+// position j ^ (r & 7) (128-byte swizzle).  The code tile arrived with the
+// same swizzle on its single 128-byte row, so neither side has bank
+// conflicts.  A code becomes a float exactly: biased by 128 it is the low
+// mantissa byte of 2^23 (one byte permute), and subtracting 2^23 + 128 is
+// exact.
+__device__ __forceinline__ void convert_row(uint32_t src_row, uint32_t dst_row, uint32_t sw,
+                                            float scale) {
+  const uint64_t sc2 = f2(scale, scale);
+  const uint64_t off2 = f2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {  // 16 codes: dims 16q .. 16q + 15
+    uint32_t w[4];
+    lds128(src_row + (((uint32_t)q ^ sw) << 4), w);
+    uint32_t out[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t b = w[i] ^ 0x80808080u;
+      const float c0 = __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7540));
+      const float c1 = __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7541));
+      const float c2 = __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7542));
+      const float c3 = __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7543));
+      const float2 v01 = unf2(mul2(add2(f2(c0, c1), off2), sc2));
+      const float2 v23 = unf2(mul2(add2(f2(c2, c3), off2), sc2));
+      out[2 * i] = pack_bf16x2(v01.x, v01.y);
+      out[2 * i + 1] = pack_bf16x2(v23.x, v23.y);
+    }
+    const uint32_t c0 = 2u * q, c1 = 2u * q + 1u;  // 8-dim chunks of the output row
+    sts128(dst_row + (c0 >> 3) * kHalfBytes + (((c0 & 7u) ^ sw) << 4), out);
+    sts128(dst_row + (c1 >> 3) * kHalfBytes + (((c1 & 7u) ^ sw) << 4), out + 4);
+  }
+}
 
 // Walks this block's key tiles as (span, tile within the span).  Dense mode
 // visits the global tiles [g0, g1) in order (all of them without a key
@@ -377,9 +468,17 @@ struct TileWalk {
   }
 };
 
-template <bool kSparse>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kSparse, bool kI8>
+__global__ void __launch_bounds__(Cfg<kI8>::kThreads, 1)
 attention_kernel(const __grid_constant__ AttnArgs p) {
+  using C = Cfg<kI8>;
+  constexpr int kStages = C::kStages;
+  constexpr uint32_t kOffQ = C::kOffQ, kOffKV = C::kOffKV, kOffStage = C::kOffStage,
+                     kOffBar = C::kOffBar, kOffTmemSlot = C::kOffTmemSlot, kOffAbort = C::kOffAbort;
+  constexpr int kBarQFull = C::kBarQFull, kBarKVFull = C::kBarKVFull,
+                kBarKVEmpty = C::kBarKVEmpty, kBarSFull = C::kBarSFull, kBarPFull = C::kBarPFull,
+                kBarPHalf = C::kBarPHalf, kBarOFull = C::kBarOFull, kBarDrain = C::kBarDrain,
+                kBarStFull = C::kBarStFull, kBarStEmpty = C::kBarStEmpty;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -392,6 +491,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
 
   const uint32_t sQ = base + kOffQ;
   const uint32_t sKV = base + kOffKV;
+  const uint32_t sStage = base + kOffStage;  // INT8 variant: code tiles from TMA
   auto bar = [&](int i) { return base + kOffBar + (uint32_t)i * 8u; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + kOffTmemSlot);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + kOffAbort);
@@ -409,6 +509,10 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       mbar_init(bar(kBarOFull + t), 1);
     }
     mbar_init(bar(kBarDrain), 1);
+    for (int st = 0; st < C::kStaging; ++st) {
+      mbar_init(bar(kBarStFull + st), 1);
+      mbar_init(bar(kBarStEmpty + st), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -445,7 +549,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
     while (w.next(&s_, &kt_, &bad_)) ++n_kv;
   }
 
-  if (warp == kProducerWarp) {
+  auto role_producer = [&]() {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_q = l2_policy_evict_first();
@@ -456,6 +560,10 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           tma_load_2d(sQ + i * kTileBytes + c * kHalfBytes, &p.tmap_q, bar(kBarQFull),
                       head * kHeadDim + c * 64, q_row0 + i * kBM, pol_q);
       int t = 0;
+      // INT8 variant: code tiles issued to the staging slots, the one left
+      // out by the testing hook, and the end of the ring indices that the
+      // converters fill (the INT8 span comes first).
+      int u = 0, u_skip = -1, t_i8_end = 0;
       bool ok = true;
       TileWalk<kSparse> walk(p, list, n_list, g0, g1);
       int s, kt;
@@ -463,6 +571,26 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       while (ok && walk.next(&s, &kt, &bad)) {
         {
           for (int which = 0; which < 2; ++which, ++t) {
+            if (kI8 && s == 0) {
+              // INT8 tile: its codes go to a staging slot; the converter
+              // warpgroup fills ring slot t from there.
+              const int st = u & 1;
+              const uint32_t sph = (uint32_t)(u >> 1) & 1u;
+              t_i8_end = t + 1;
+              if (t == p.testing_skip_load) {
+                u_skip = u++;
+                continue;
+              }
+              if (!wait_phase(bar(kBarStEmpty + st), sph ^ 1u, ctl)) {
+                ok = false;
+                break;
+              }
+              mbar_expect_tx(bar(kBarStFull + st), kCodeTileBytes);
+              tma_load_2d(sStage + st * kCodeTileBytes, which == 0 ? &p.tmap_k[0] : &p.tmap_v[0],
+                          bar(kBarStFull + st), head * kHeadDim, kt * kBN, pol_kv);
+              ++u;
+              continue;
+            }
             // Testing hook: leave one load out so that a consumer wait runs
             // out of time (exercises the bounded-wait abort path).
             if (t == p.testing_skip_load) continue;
@@ -481,14 +609,19 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
         }
       }
       if (bad && p.dev_err != nullptr) atomicOr(p.dev_err, NOMAS_DEVERR_BAD_TILE_INDEX);
-      // Teardown: wait until every load this lane issued has landed.
+      // Teardown: wait until every load this lane issued has landed (ring
+      // slots the converters fill are theirs, not this lane's).
       drain_phase(bar(kBarQFull), 0, p.wait_limit_ns);
-      for (int u = (t > kStages ? t - kStages : 0); u < t; ++u)
-        if (u != p.testing_skip_load)
-          drain_phase(bar(kBarKVFull + u % kStages), (uint32_t)(u / kStages) & 1u, p.wait_limit_ns);
+      for (int v = max(t - kStages, t_i8_end); v < t; ++v)
+        if (v != p.testing_skip_load)
+          drain_phase(bar(kBarKVFull + v % kStages), (uint32_t)(v / kStages) & 1u, p.wait_limit_ns);
+      for (int v = max(u - 2, 0); v < u; ++v)
+        if (v != u_skip)
+          drain_phase(bar(kBarStFull + (v & 1)), (uint32_t)(v >> 1) & 1u, p.wait_limit_ns);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  };
+  auto role_mma = [&]() {
     // ------------------------------------------------------------------ MMA
     if (lane == 0 && n_kv > 0) {
       const uint32_t tS[2] = {tmem_base + 0u, tmem_base + 128u};
@@ -551,7 +684,50 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       drain_phase(bar(kBarDrain), 0, p.wait_limit_ns);
     }
     __syncwarp();
-  } else {
+  };
+  auto role_convert = [&]() {
+    // ---------------------------------------------------------- converters
+    // INT8 variant only: warps 10-11 have no role; warps 12-15 (one per
+    // sub-partition) dequantise the INT8 span's code tiles into the ring,
+    // thread r handling key row r of every tile.
+    if constexpr (kI8) {
+      if (warp >= kConvWarp0) {
+        const int r = (int)threadIdx.x - kConvWarp0 * 32;
+        const uint32_t sw = (uint32_t)(r & 7);
+        int t = 0, u = 0;
+        bool ok = true;
+        TileWalk<kSparse> walk(p, list, n_list, g0, g1);
+        int s, kt;
+        bool bad = false;
+        while (ok && walk.next(&s, &kt, &bad)) {
+          if (s != 0) break;  // the INT8 span comes first; the producer loads the rest
+          const int64_t key = (int64_t)kt * kBN + r;
+          const bool in_span = key < p.span_len[0];
+          for (int which = 0; which < 2; ++which, ++t, ++u) {
+            const float scale = in_span ? __ldg(p.i8_scale[which] + key * kHeads + head) : 0.f;
+            const int st = u & 1;
+            const int slot = t % kStages;
+            const bool got =
+                wait_phase(bar(kBarStFull + st), (uint32_t)(u >> 1) & 1u, ctl) &&
+                wait_phase(bar(kBarKVEmpty + slot), ((uint32_t)(t / kStages) & 1u) ^ 1u, ctl);
+            if (!converters_all(got)) {
+              ok = false;
+              break;
+            }
+            convert_row(sStage + st * kCodeTileBytes + r * 128, sKV + slot * kTileBytes + r * 128,
+                        sw, scale);
+            fence_proxy_async_smem();
+            converters_sync();
+            if (r == 0) {
+              mbar_arrive(bar(kBarKVFull + slot));
+              mbar_arrive(bar(kBarStEmpty + st));
+            }
+          }
+        }
+      }
+    }
+  };
+  auto role_softmax = [&]() {
     // -------------------------------------------------------------- softmax
     const int tile = warp >> 2;
     const int quarter = warp & 3;
@@ -764,17 +940,48 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       }
       if (lse_out != nullptr && row < p.n_q)
         lse_out[(int64_t)head * p.n_q + row] = (m + log2f(l)) * 0.69314718055994531f;
-    } else if (ok && n_kv == 0) {
+    } else {
       // No key selected for this block (a sparse list with no valid entry):
-      // the empty sums give O = 0 and LSE = -inf.
+      // the empty sums give O = 0 and LSE = -inf.  A block that aborted (a
+      // wait ran out) marks its rows NaN instead, so that nothing downstream
+      // -- a merge of key-split or key-sharded partials in particular -- can
+      // take earlier contents of the buffers for this block's result.
+      const bool empty = ok && n_kv == 0;
+      const uint32_t fill = empty ? 0u : 0x7FC07FC0u;  // bf16 0 or quiet NaN pairs
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       if (row < p.n_q) {
         uint4 *dst = reinterpret_cast<uint4 *>(o_out + row * kRowElems + head * kHeadDim);
 #pragma unroll
-        for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-        if (lse_out != nullptr) lse_out[(int64_t)head * p.n_q + row] = -INFINITY;
+        for (int v = 0; v < 16; ++v) dst[v] = make_uint4(fill, fill, fill, fill);
+        if (lse_out != nullptr) lse_out[(int64_t)head * p.n_q + row] = empty ? -INFINITY : NAN;
       }
     }
+  };
+
+  if constexpr (kI8) {
+    // setmaxnreg is warpgroup-collective: the two softmax warpgroups (warps
+    // 0-7) raise their registers at one instruction, the producer/MMA and
+    // converter warpgroups (warps 8-15) lower theirs at another, before the
+    // roles diverge.
+    if (warp < 8) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kI8SoftmaxRegs));
+      role_softmax();
+    } else {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kI8OtherRegs));
+      if (warp == kProducerWarp)
+        role_producer();
+      else if (warp == kMmaWarp)
+        role_mma();
+      else
+        role_convert();
+    }
+  } else {
+    if (warp == kProducerWarp)
+      role_producer();
+    else if (warp == kMmaWarp)
+      role_mma();
+    else
+      role_softmax();
   }
 
   tc_fence_before();
@@ -802,20 +1009,32 @@ __global__ void attention_empty_kernel(uint16_t *o, float *lse, int64_t n_q) {
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   // The shared-memory opt-in is a per-device function attribute.  Several
   // host threads may make their first call on a device at once: the
-  // attribute calls are idempotent, and the flag is atomic.
-  static std::atomic<bool> attr_set[64];
+  // attribute calls are idempotent, and the flag is atomic.  The INT8
+  // variant's register split is only safe when the kernel was compiled to
+  // exactly the launch allocation it assumes (otherwise a warpgroup's raise
+  // could wait for registers that never come): checked here, before its
+  // first launch on the device, and refused otherwise.
+  static std::atomic<int> attr_state[64];  // 0 unset, 1 set, 2 set but INT8 refused
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(attention_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  int state = attr_state[dev].load(std::memory_order_acquire);
+  if (state == 0) {
+    e = cudaFuncSetAttribute(attention_kernel<false, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemAlloc);
+    e = cudaFuncSetAttribute(attention_kernel<true, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<false>::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    attr_set[dev].store(true, std::memory_order_release);
+    e = cudaFuncSetAttribute(attention_kernel<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<true>::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, attention_kernel<false, true>);
+    if (e != cudaSuccess) return e;
+    state = (fa.numRegs == kI8LaunchRegs && fa.maxThreadsPerBlock >= Cfg<true>::kThreads) ? 1 : 2;
+    attr_state[dev].store(state, std::memory_order_release);
   }
   const int64_t q_blocks = ((int64_t)a.n_q + kQTiles * kBM - 1) / (kQTiles * kBM);
   if (q_blocks <= 0) return cudaSuccess;
@@ -824,10 +1043,16 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
       (a.kv_splits > 1 && (a.tile_list != nullptr || a.lse == nullptr)))
     return cudaErrorInvalidValue;
   dim3 grid((unsigned)q_blocks, kHeads, (unsigned)a.kv_splits);
-  if (a.tile_list != nullptr)
-    attention_kernel<true><<<grid, kThreads, kSmemAlloc, stream>>>(a);
-  else
-    attention_kernel<false><<<grid, kThreads, kSmemAlloc, stream>>>(a);
+  if (a.i8) {
+    if (a.tile_list != nullptr) return cudaErrorInvalidValue;
+    if (state != 1) return cudaErrorInvalidKernelImage;
+    attention_kernel<false, true><<<grid, Cfg<true>::kThreads, Cfg<true>::kSmemAlloc, stream>>>(a);
+  } else if (a.tile_list != nullptr) {
+    attention_kernel<true, false><<<grid, Cfg<false>::kThreads, Cfg<false>::kSmemAlloc, stream>>>(a);
+  } else {
+    attention_kernel<false, false><<<grid, Cfg<false>::kThreads, Cfg<false>::kSmemAlloc, stream>>>(
+        a);
+  }
   return cudaGetLastError();
 }
 

@@ -78,19 +78,26 @@ merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
     const int h = threadIdx.x >> 4, rr = threadIdx.x & 15;
     const int64_t row = row0 + rr;
     float *w = w_s + rr * kWRow + h;
+    // A NaN LSE marks a partial whose attention block aborted: the merged
+    // row becomes NaN (weights and LSE), never a merge of the other parts.
     float m = -INFINITY;
+    bool bad = false;
     if (row < row_end)
-      for (int r = 0; r < n_parts; ++r) m = fmaxf(m, parts.lse_at(r, h, row));
+      for (int r = 0; r < n_parts; ++r) {
+        const float x = parts.lse_at(r, h, row);
+        bad |= isnan(x);
+        m = fmaxf(m, x);
+      }
     float total = 0.f;
     for (int r = 0; r < n_parts; ++r) {
       const float e = m == -INFINITY ? 0.f : expf(parts.lse_at(r, h, row) - m);
       w[r * kWPlane] = e;
       total += e;
     }
-    const float inv = total > 0.f ? 1.f / total : 0.f;
+    const float inv = bad ? NAN : (total > 0.f ? 1.f / total : 0.f);
     for (int r = 0; r < n_parts; ++r) w[r * kWPlane] *= inv;
     if (row < row_end) {
-      const float l = total > 0.f ? m + logf(total) : -INFINITY;
+      const float l = bad ? NAN : (total > 0.f ? m + logf(total) : -INFINITY);
       for (int k = 0; k < outs.n; ++k)
         if (outs.lse[k] != nullptr) outs.lse[k][(int64_t)h * n_q + row] = l;
     }

@@ -15,11 +15,17 @@
 // shares it: calls that overlap on the GPU (two streams, or two host threads)
 // race on it and must be serialised by the caller.  Each call overwrites
 // every byte it reads (each partial output row and LSE is written by its CTA
-// before the merge reads it), so nothing has to start at zero.
+// before the merge reads it; a CTA whose pipeline wait ran out writes NaN
+// rows, which the merge turns into NaN output rows), so nothing has to start
+// at zero and no earlier call's contents can reach an output.
 //
-// The first call on each device looks up the array's device address
-// (cudaGetSymbolAddress, with that device current) and keeps it; make that
-// first call before any stream capture begins.
+// The array's device address is asked of the runtime (cudaGetSymbolAddress,
+// with the device current) on every call made outside stream capture, and
+// kept per device.  A call made while its stream is capturing uses the kept
+// address instead, since the lookup may load the module, which capture does
+// not allow: make one call on the device before capturing, and another after
+// the device's primary context has been reset (cudaDeviceReset), which moves
+// the array.
 #include <cstdio>
 #include <mutex>
 
@@ -40,18 +46,31 @@ constexpr int kMaxDevices = 64;
 void *g_scratch_ptr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-cudaError_t scratch_address(void **out) {
+// True unless `stream` is known not to be capturing.  Asking about the legacy
+// stream while another stream captures in global mode is itself an error;
+// that counts as capturing.
+bool maybe_capturing(cudaStream_t stream) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return true;
+  }
+  return st != cudaStreamCaptureStatusNone;
+}
+
+cudaError_t scratch_address(cudaStream_t stream, void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (!maybe_capturing(stream)) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_split_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
   }
+  if (g_scratch_ptr[dev] == nullptr) return cudaErrorStreamCaptureUnsupported;
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
 }
@@ -73,10 +92,14 @@ extern "C" nomas_status nomas_segment_attention_split_noalloc(
   }
   void *scratch = nullptr;
   if (need > 0) {
-    const cudaError_t e = scratch_address(&scratch);
+    const cudaError_t e = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
     if (e != cudaSuccess) {
-      char msg[200];
-      snprintf(msg, sizeof(msg), "device address of the built-in scratch array: %s",
+      char msg[240];
+      snprintf(msg, sizeof(msg),
+               e == cudaErrorStreamCaptureUnsupported
+                   ? "device address of the built-in scratch array: not known yet on this "
+                     "device and the stream is capturing (make one call before capture)"
+                   : "device address of the built-in scratch array: %s",
                cudaGetErrorString(e));
       return nomas::report_error(NOMAS_ERR_CUDA, msg);
     }

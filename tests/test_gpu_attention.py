@@ -202,11 +202,14 @@ def test_wait_timeout_is_reported_and_context_survives():
     sd = [(k.cuda(), v.cuda()) for k, v in spans]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     o = torch.full((112, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
-    nm.segment_attention(q.cuda(), sd, o=o, dev_err=err, wait_limit_ns=50_000_000,
+    lse = torch.full((16 * 112,), 7.0, dtype=torch.float32, device="cuda")
+    nm.segment_attention(q.cuda(), sd, o=o, lse=lse, dev_err=err, wait_limit_ns=50_000_000,
                          testing_skip_kv_load=3)
     torch.cuda.synchronize()
     assert int(err.item()) == nm.DEVERR_WAIT_TIMEOUT
-    assert torch.all(o == 7.0)  # aborted blocks write no output
+    # every block leaves out its fourth load and aborts: its rows are NaN, so
+    # nothing earlier in the buffers can pass for a result
+    assert torch.all(torch.isnan(o)) and torch.all(torch.isnan(lse))
     # the same context still computes correct results
     _check(q, spans, what="after timeout")
 

@@ -32,6 +32,30 @@ def test_merge_kernel_matches_oracle_formula(r, n_q):
     assert np.allclose(got_l[fin], want_l[fin], atol=1e-5)
 
 
+def test_merge_nan_partial_poisons_only_its_rows():
+    # A NaN LSE marks a partial whose attention block aborted: those (row,
+    # head) pairs come out NaN, never as a merge of the remaining parts; every
+    # other row is the plain merge.
+    r, n_q = 4, 300
+    o_parts = randn_bf16((r, n_q, 16, 128), 8)
+    lse_parts = torch.randn((r, 16, n_q), generator=torch.Generator().manual_seed(4)) * 3
+    lse_parts[2, 5, 100:120] = float("nan")
+    lse = torch.empty(16 * n_q, dtype=torch.float32, device="cuda")
+    o = nm.attention_merge(o_parts.cuda(), lse_parts.cuda(), lse=lse)
+    torch.cuda.synchronize()
+    got_o, got_l = f64(o), lse.view(16, n_q).cpu().double().numpy()
+    bad = np.zeros((n_q, 16), dtype=bool)
+    bad[100:120, 5] = True
+    assert np.all(np.isnan(got_o[bad])) and np.all(np.isnan(got_l.T[bad]))
+    clean = lse_parts.clone()
+    clean[2, 5, 100:120] = 0.0
+    want_o, want_l = oracle.merge_partials(f64(o_parts), clean.double().numpy())
+    assert not np.any(np.isnan(got_o[~bad]))
+    assert_bf16_rounding(np.where(bad[:, :, None], 0.0, got_o),
+                         np.where(bad[:, :, None], 0.0, want_o), what="merged O, clean rows")
+    assert np.allclose(got_l.T[~bad], want_l.T[~bad], atol=1e-5)
+
+
 @pytest.mark.parametrize("cuts", [[0, 1000, 2500, 4000], [0, 0, 4000], [0, 1, 3999, 4000]])
 def test_sharded_keys_merge_to_full_attention(cuts):
     q = randn_bf16((700, 16, 128), 1)

@@ -8,9 +8,11 @@ For them nomas_segment_attention_split_noalloc runs the key-split attention
 on a scratch array built into the library instead of caller memory.
 
 Through the C ABI, two calls in a row (with different shapes, so the second
-reads nothing the first left behind) must give the results of the existing
-entry points, and a request larger than the array must be refused before
-anything runs.  This file is collected last on purpose, and passes alone in
+reads nothing the first left behind) must give, bit for bit, the result of
+the existing key-split entry point with caller scratch (the same kernel, the
+same split, the same stream), plain attention's result within the parity
+bar, and the fp64 oracle's within the same bar; a request larger than the
+array must be refused before anything runs.  This file is collected last on purpose, and passes alone in
 a fresh process as well as after every other test.
 """
 import ctypes
@@ -20,8 +22,9 @@ import pytest
 import torch
 
 import kv_cached_segment_b200 as nm
+import oracle
 from seeded_inputs import randn_bf16
-from tests._util import assert_close, f64
+from tests._util import assert_close, bits, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -65,9 +68,15 @@ def test_noalloc_split_matches_the_existing_entry_points_on_two_calls_in_a_row()
         torch.cuda.synchronize()
         assert st == nm.NOMAS_OK, lib.nomas_last_error().decode()
         assert int(err.item()) == 0
-        assert_close(f64(o), f64(o_ref), what=f"no-alloc vs caller scratch, call {seed}")
+        # same kernel, same split, same stream: identical bits
+        assert np.array_equal(bits(o), bits(o_ref)), f"no-alloc vs caller scratch, call {seed}"
+        assert np.array_equal(lse.cpu().numpy().view(np.uint32),
+                              lse_ref.cpu().numpy().view(np.uint32))
         assert_close(f64(o), f64(o_plain), what=f"no-alloc vs plain attention, call {seed}")
-        assert np.allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), atol=2e-2)
+        o_or, l_or = oracle.attention(f64(q), [(f64(k), f64(v)) for k, v in spans])
+        assert_close(f64(o), o_or, what=f"no-alloc vs oracle, call {seed}")
+        assert_close(lse.view(16, n_q).cpu().double().numpy(), l_or,
+                     what=f"no-alloc LSE vs oracle, call {seed}")
 
 
 def test_noalloc_refuses_more_than_its_array():
