@@ -11,9 +11,11 @@ Entry points (same names as the C ABI, without the ``nomas_`` prefix):
 - ``kvcache_append`` / ``kvcache_append_i8``: rotate the segment's K into a
   bf16 or INT8 cache (V copied or quantised), optionally Q too;
 - ``kvcache_select``: gather latent frames of a bf16 or INT8 cache into a
-  bf16 window;
+  bf16 window, or of an INT8 cache into an INT8 window;
 - ``segment_attention`` / ``segment_attention_sparse``: attention of the
-  query rows over up to four key/value spans, all tiles or listed tiles;
+  query rows over up to four key/value spans, all tiles or listed tiles; a
+  first span that is an INT8 ``I8Span`` (``KVCacheI8.span()``) is read as
+  codes and scales and dequantised inside the kernel;
 - ``attention_merge``: combine partial (O, LSE) over disjoint key shards;
 - ``temporal_context_frames``: the power-spaced history frame picker (host).
 
@@ -71,6 +73,8 @@ EXPORTED_SYMBOLS = (
     "nomas_segment_attention_scratch_bytes",
     "nomas_attention_merge_peers",
     "nomas_segment_attention_to_owners",
+    "nomas_kvcache_select_i8_codes",
+    "nomas_segment_attention_i8",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -108,6 +112,11 @@ class _KVCacheI8(ctypes.Structure):
 
 class _KVSpan(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_int64)]
+
+
+class _KVSpanI8(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("len", ctypes.c_int64)]
 
 
 class _AttnOpts(ctypes.Structure):
@@ -173,6 +182,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_segment_attention_to_owners.restype = ctypes.c_int
     lib.nomas_segment_attention_to_owners.argtypes = [P, I64, ctypes.POINTER(_KVSpan), I32, I32, P,
                                                       P, P, I32, F32, I32, I32, P, P]
+    lib.nomas_kvcache_select_i8_codes.restype = ctypes.c_int
+    lib.nomas_kvcache_select_i8_codes.argtypes = [ctypes.POINTER(_KVCacheI8), P, I32, I32,
+                                                  ctypes.POINTER(_KVCacheI8), P, P]
+    lib.nomas_segment_attention_i8.restype = ctypes.c_int
+    lib.nomas_segment_attention_i8.argtypes = [P, I64, ctypes.POINTER(_KVSpanI8),
+                                               ctypes.POINTER(_KVSpan), I32, P, P, F32, I32, I32,
+                                               P, ctypes.POINTER(_AttnOpts), P]
     lib.nomas_temporal_context_frames.restype = ctypes.c_int
     lib.nomas_temporal_context_frames.argtypes = [I32, I32, F32, P, I32, P]
     _lib = lib
@@ -305,6 +321,39 @@ class KVCacheI8:
     def capacity(self) -> int:
         return self._c.capacity
 
+    @property
+    def tokens_per_frame(self) -> int:
+        return self._c.tokens_per_frame
+
+    def span(self, start: int = 0, stop: int | None = None) -> "I8Span":
+        """Rows [start, stop) (default: all valid rows) as an INT8 key/value span."""
+        stop = self.len if stop is None else stop
+        return I8Span(self.k[start:stop], self.v[start:stop], self.k_scale[start:stop],
+                      self.v_scale[start:stop])
+
+
+@dataclass
+class I8Span:
+    """INT8 rows of keys and values: codes [N][16][128] int8, scales [N][16] fp32."""
+
+    k: torch.Tensor
+    v: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+
+    def _c(self) -> _KVSpanI8:
+        n = self.k.shape[0]
+        for t, name in ((self.k, "k"), (self.v, "v")):
+            if t.dtype != torch.int8 or not t.is_cuda or not t.is_contiguous() or \
+                    t.dim() != 3 or t.shape != (n, HEADS, HEAD_DIM):
+                raise TypeError(f"INT8 span {name} must be contiguous CUDA int8 [N][16][128]")
+        for t, name in ((self.k_scale, "k_scale"), (self.v_scale, "v_scale")):
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or \
+                    t.shape != (n, HEADS):
+                raise TypeError(f"INT8 span {name} must be contiguous CUDA fp32 [N][16]")
+        ptr = (lambda t: t.data_ptr() if n else None)  # noqa: E731
+        return _KVSpanI8(ptr(self.k), ptr(self.v), ptr(self.k_scale), ptr(self.v_scale), n)
+
 
 def kvcache_append_i8(cache: KVCacheI8, k_seg, v_seg, q_in=None, q_out=None,
                       layout: SegLayout | None = None, cfg: RopeConfig | None = None,
@@ -373,11 +422,13 @@ def temporal_context_frames(n_past: int, budget: int = 18, gamma: float = 2.0) -
     return [int(out[i]) for i in range(n_out.value)]
 
 
-def kvcache_select(src, frame_idx, window: KVCache, dev_err=None, stream=None) -> None:
-    """Gathers the listed latent frames of ``src`` into the bf16 ``window``.
+def kvcache_select(src, frame_idx, window, dev_err=None, stream=None) -> None:
+    """Gathers the listed latent frames of ``src`` into ``window``.
 
-    A bf16 ``src`` is copied bit for bit; an INT8 ``src`` (KVCacheI8) is
-    dequantised (code * scale, rounded to bf16).
+    A bf16 ``src`` is copied bit for bit into a bf16 window.  An INT8 ``src``
+    (KVCacheI8) is either dequantised into a bf16 window (code * scale,
+    rounded once to bf16) or, into an INT8 window, copied as codes and
+    scales bit for bit.
     """
     lib = load_library()
     if isinstance(frame_idx, torch.Tensor) and frame_idx.is_cuda:
@@ -391,7 +442,12 @@ def kvcache_select(src, frame_idx, window: KVCache, dev_err=None, stream=None) -
         ptr = ctypes.cast(arr, ctypes.c_void_p).value
     if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
         raise TypeError("dev_err must be a CUDA int32 tensor")
-    fn = lib.nomas_kvcache_select_i8 if isinstance(src, KVCacheI8) else lib.nomas_kvcache_select
+    if isinstance(window, KVCacheI8):
+        if not isinstance(src, KVCacheI8):
+            raise TypeError("an INT8 window needs an INT8 source cache")
+        fn = lib.nomas_kvcache_select_i8_codes
+    else:
+        fn = lib.nomas_kvcache_select_i8 if isinstance(src, KVCacheI8) else lib.nomas_kvcache_select
     _check(fn(ctypes.byref(src._c), ptr, n, on_dev, ctypes.byref(window._c), _ptr(dev_err),
               _stream(stream)))
     del keep
@@ -443,6 +499,11 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         raise ValueError("lse must be a contiguous CUDA fp32 tensor of heads * n_q elements")
     if len(spans) > MAX_SPANS:
         raise ValueError(f"at most {MAX_SPANS} spans")
+    history = None
+    if spans and isinstance(spans[0], I8Span):
+        history, spans = spans[0]._c(), list(spans[1:])
+        if kv_splits not in (1, "1"):
+            raise ValueError("an INT8 history span takes kv_splits=1")
     arr = (_KVSpan * max(1, len(spans)))()
     for i, (k, v) in enumerate(spans):
         nk = _rows(k, f"span {i} k")
@@ -455,7 +516,13 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         sm = torch.cuda.get_device_properties(q.device).multi_processor_count
         kv_splits = auto_kv_splits(n_q, [int(k.shape[0]) for k, _ in spans], sm)
     kv_splits = int(kv_splits)
-    if kv_splits > 1:
+    if history is not None:
+        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load))
+        _check(lib.nomas_segment_attention_i8(_ptr(q), n_q, ctypes.byref(history), arr, len(spans),
+                                              _ptr(o), _ptr(lse), float(softmax_scale), HEADS,
+                                              HEAD_DIM, _ptr(dev_err), ctypes.byref(opts),
+                                              _stream(stream)))
+    elif kv_splits > 1:
         if wait_limit_ns or testing_skip_kv_load != -1:
             raise ValueError("kv_splits > 1 takes no wait_limit_ns / testing_skip_kv_load")
         if stream is not None and not isinstance(stream, torch.cuda.Stream):

@@ -146,6 +146,23 @@ nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows) {
   return NOMAS_OK;
 }
 
+// 2-D view of a [rows][16][128] int8 code tensor: inner extent 2048 bytes,
+// row pitch 2048 B; box = 128 codes (one head, one swizzle span) x 128 rows.
+nomas_status codes_map(CUtensorMap *m, const void *ptr, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {(cuuint64_t)kRowElems, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kRowElems};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NOMAS_OK;
+}
+
 // A bf16 or INT8 layer cache seen by the append path.
 struct CacheView {
   void *k, *v;
@@ -329,7 +346,8 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               float softmax_scale, int32_t heads, int32_t head_dim,
                               int32_t *dev_err, const nomas_attention_opts *opts,
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
-                              const struct OwnerRouting *routing, void *stream);
+                              const struct OwnerRouting *routing, void *stream,
+                              const nomas_kv_span_i8 *i8_span = nullptr);
 
 // Destination of owner-routed partial outputs (see AttnArgs::n_owners).
 struct OwnerRouting {
@@ -443,6 +461,93 @@ nomas_status nomas_kvcache_select_i8(const nomas_kvcache_i8 *src, const int32_t 
                  src->heads, src->head_dim, true};
   return select_common(view, src->tokens_per_frame, frame_idx, n_frames, idx_on_device, window,
                        dev_err, stream);
+}
+
+nomas_status nomas_kvcache_select_i8_codes(const nomas_kvcache_i8 *src, const int32_t *frame_idx,
+                                           int32_t n_frames, int32_t idx_on_device,
+                                           nomas_kvcache_i8 *window, int32_t *dev_err,
+                                           void *stream) {
+  const ApiRange nvtx_range("nomas_kvcache_select_i8_codes");
+  if (src == nullptr || window == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "src/window is NULL");
+  nomas_status st = check_shape(src->heads, src->head_dim);
+  if (st != NOMAS_OK) return st;
+  if ((st = check_shape(window->heads, window->head_dim)) != NOMAS_OK) return st;
+  const int64_t P = src->tokens_per_frame;
+  if (P <= 0) return fail(NOMAS_ERR_INVALID_ARG, "src tokens_per_frame <= 0");
+  if (n_frames < 0) return fail(NOMAS_ERR_INVALID_ARG, "n_frames < 0");
+  if (src->len < 0 || src->len > src->capacity || window->capacity < 0)
+    return fail(NOMAS_ERR_INVALID_ARG, "src len/capacity inconsistent");
+  const int64_t rows = (int64_t)n_frames * P;
+  if (rows > window->capacity)
+    return fail(NOMAS_ERR_CAPACITY, "window capacity %lld < %d frames x %lld rows",
+                (long long)window->capacity, n_frames, (long long)P);
+  if (n_frames > 0) {
+    if (frame_idx == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "frame_idx is NULL");
+    const void *ptrs[8] = {src->k, src->v, src->k_scale, src->v_scale,
+                           window->k, window->v, window->k_scale, window->v_scale};
+    for (const void *q : ptrs)
+      if (q == nullptr || !aligned16(q))
+        return fail(NOMAS_ERR_INVALID_ARG,
+                    "INT8 caches' codes and scales must be non-NULL and 16-byte aligned");
+    const int64_t scb = src->len * kRowElems, sscb = src->len * kHeads * 4;
+    const int64_t wcb = rows * kRowElems, wscb = rows * kHeads * 4;
+    const int64_t ssz[4] = {scb, scb, sscb, sscb}, wsz[4] = {wcb, wcb, wscb, wscb};
+    for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 4; ++j)
+        if (overlap(ptrs[i], ssz[i], ptrs[4 + j], wsz[j]) ||
+            (j > i && overlap(ptrs[4 + i], wsz[i], ptrs[4 + j], wsz[j])))
+          return fail(NOMAS_ERR_INVALID_ARG, "window overlaps the source cache or itself");
+  }
+  const int64_t n_src_frames = src->len / P;
+  if (idx_on_device && n_frames > 0 && dev_err == nullptr)
+    return fail(NOMAS_ERR_INVALID_ARG, "dev_err is required for a device-resident frame list");
+  if (!idx_on_device) {
+    for (int32_t j = 0; j < n_frames; ++j)
+      if (frame_idx[j] < 0 || frame_idx[j] >= n_src_frames)
+        return fail(NOMAS_ERR_INDEX, "frame_idx[%d] = %d outside [0, %lld)", j, frame_idx[j],
+                    (long long)n_src_frames);
+  }
+  // Codes and scales are plain byte runs per frame: the bit-copy gather of
+  // the bf16 path moves them, once for the codes and once for the scales.
+  const int chunk = idx_on_device ? 65535 : kSelectHostFramesPerLaunch;
+  SelectHostList hl;
+  for (int32_t f0 = 0; f0 < n_frames; f0 += chunk) {
+    const int32_t nf = (n_frames - f0) < chunk ? (n_frames - f0) : chunk;
+    if (!idx_on_device) std::memcpy(hl.idx, frame_idx + f0, sizeof(int32_t) * nf);
+    for (int part = 0; part < 2; ++part) {
+      SelectArgs a{};
+      a.src_k = static_cast<const uint16_t *>(part == 0 ? src->k : (const void *)src->k_scale);
+      a.src_v = static_cast<const uint16_t *>(part == 0 ? src->v : (const void *)src->v_scale);
+      a.dst_k = static_cast<uint16_t *>(part == 0 ? window->k : (void *)window->k_scale);
+      a.dst_v = static_cast<uint16_t *>(part == 0 ? window->v : (void *)window->v_scale);
+      a.idx_dev = idx_on_device ? frame_idx : nullptr;
+      // report a bad device index once, from the codes' launch
+      a.dev_err = part == 0 ? dev_err : nullptr;
+      a.frame_vecs = P * (part == 0 ? kRowElems : kHeads * 4) / 16;
+      a.n_src_frames = n_src_frames;
+      a.first_frame = f0;
+      a.n_frames = nf;
+      const cudaError_t e =
+          launch_select(a, idx_on_device ? nullptr : &hl, static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e, "select launch");
+    }
+  }
+  window->tokens_per_frame = (int32_t)P;
+  window->len = rows;
+  return ok();
+}
+
+nomas_status nomas_segment_attention_i8(const void *q, int64_t n_q,
+                                        const nomas_kv_span_i8 *history,
+                                        const nomas_kv_span *spans, int32_t n_spans, void *o,
+                                        float *lse, float softmax_scale, int32_t heads,
+                                        int32_t head_dim, int32_t *dev_err,
+                                        const nomas_attention_opts *opts, void *stream) {
+  const ApiRange nvtx_range("nomas_segment_attention_i8");
+  if (history == nullptr) return fail(NOMAS_ERR_INVALID_ARG, "history is NULL");
+  return attention_common(q, n_q, spans, n_spans, nullptr, nullptr, 0, o, lse, softmax_scale,
+                          heads, head_dim, dev_err, opts, 1, nullptr, 0, nullptr, stream,
+                          history);
 }
 
 nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, int32_t n_parts,
@@ -624,9 +729,16 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               float softmax_scale, int32_t heads, int32_t head_dim,
                               int32_t *dev_err, const nomas_attention_opts *opts,
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
-                              const OwnerRouting *routing, void *stream) {
+                              const OwnerRouting *routing, void *stream,
+                              const nomas_kv_span_i8 *i8_span) {
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
+  const bool i8 = i8_span != nullptr && i8_span->len != 0;
+  if (i8_span != nullptr && (i8_span->len < 0 || i8_span->len > 0x7fff0000LL))
+    return fail(NOMAS_ERR_INVALID_ARG, "INT8 history length out of range");
+  if (i8 && (n_spans + 1 > kMaxSpans))
+    return fail(NOMAS_ERR_UNSUPPORTED, "at most %d key/value spans with the INT8 history (got %d)",
+                kMaxSpans - 1, n_spans);
   if (kv_splits < 1 || kv_splits > NOMAS_MAX_MERGE_PARTS)
     return fail(NOMAS_ERR_INVALID_ARG, "kv_splits must be in [1, %d] (got %d)",
                 NOMAS_MAX_MERGE_PARTS, kv_splits);
@@ -658,6 +770,30 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   }
   AttnArgs a{};
   int n_used = 0;
+  if (i8) {
+    // span 0: the INT8 history (codes through TMA, scales read by the kernel)
+    const nomas_kv_span_i8 &h = *i8_span;
+    if (h.k == nullptr || h.v == nullptr || h.k_scale == nullptr || h.v_scale == nullptr ||
+        !aligned16(h.k) || !aligned16(h.v) || !aligned16(h.k_scale) || !aligned16(h.v_scale))
+      return fail(NOMAS_ERR_INVALID_ARG,
+                  "INT8 history codes and scales must be non-NULL and 16-byte aligned");
+    const int64_t cb = h.len * kRowElems, scb = h.len * kHeads * 4;
+    const void *parts[4] = {h.k, h.v, h.k_scale, h.v_scale};
+    const int64_t sizes[4] = {cb, cb, scb, scb};
+    for (int i = 0; i < 4; ++i)
+      if (overlap(parts[i], sizes[i], o, qb) ||
+          (lse != nullptr && overlap(parts[i], sizes[i], lse, n_q * kHeads * 4)) ||
+          overlap(parts[i], sizes[i], scratch, sb))
+        return fail(NOMAS_ERR_INVALID_ARG, "INT8 history overlaps an output or the scratch");
+    if ((st = codes_map(&a.tmap_k[0], h.k, h.len)) != NOMAS_OK) return st;
+    if ((st = codes_map(&a.tmap_v[0], h.v, h.len)) != NOMAS_OK) return st;
+    a.span_len[0] = h.len;
+    a.tile_base[1] = (int32_t)((h.len + 127) / 128);
+    a.i8 = 1;
+    a.i8_scale[0] = h.k_scale;
+    a.i8_scale[1] = h.v_scale;
+    n_used = 1;
+  }
   for (int s = 0; s < n_spans; ++s) {
     const nomas_kv_span &sp = spans[s];
     if (sp.len < 0 || sp.len > 0x7fff0000LL)
@@ -737,6 +873,9 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
     a.testing_skip_load = opts->testing_skip_kv_load;
   }
   cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidKernelImage && a.i8)
+    return fail(NOMAS_ERR_CUDA, "INT8 attention kernel not compiled to %d registers per thread at "
+                "launch; refusing to run its register split", 128);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (kv_splits > 1) {
     e = launch_merge(part_o, part_lse, kv_splits, n_q, static_cast<uint16_t *>(o), lse,

@@ -106,6 +106,11 @@ struct AttnArgs {
   int64_t owner_row0[NOMAS_MAX_MERGE_PARTS + 1];
   uint16_t *owner_o[NOMAS_MAX_MERGE_PARTS];
   float *owner_lse[NOMAS_MAX_MERGE_PARTS];
+  // INT8 history: when i8 != 0, span 0 is INT8 codes (tmap_k[0] / tmap_v[0]
+  // map [len][16][128] int8) with fp32 scales i8_scale[0] (K) and
+  // i8_scale[1] (V), [len][16]; value = code * scale.
+  int32_t i8;
+  const float *i8_scale[2];
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,

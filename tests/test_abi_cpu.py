@@ -228,6 +228,60 @@ def test_int8_append_and_select_validation(lib):
     assert st == nm.NOMAS_ERR_INVALID_ARG
 
 
+def test_int8_window_select_validation(lib):
+    src = _cache_i8(240, 240)
+    win = _cache_i8(96, 0, tpf=0, base=FAKE + 10 ** 9)
+    idx = (ctypes.c_int32 * 2)(0, 10)   # frame 10 is outside 240 rows / 24 = 10 frames
+    st = lib.nomas_kvcache_select_i8_codes(ctypes.byref(src), idx, 2, 0, ctypes.byref(win), None,
+                                           None)
+    assert st == nm.NOMAS_ERR_INDEX and win.len == 0
+    ok_idx = (ctypes.c_int32 * 5)(0, 1, 2, 3, 4)
+    st = lib.nomas_kvcache_select_i8_codes(ctypes.byref(src), ok_idx, 5, 0, ctypes.byref(win),
+                                           None, None)
+    assert st == nm.NOMAS_ERR_CAPACITY  # 5 x 24 rows > 96
+    overl = _cache_i8(96, 0, tpf=0, base=FAKE + 240 * 2048)  # window codes on the source's V
+    st = lib.nomas_kvcache_select_i8_codes(ctypes.byref(src), ok_idx, 2, 0, ctypes.byref(overl),
+                                           None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    noscale = _cache_i8(96, 0, tpf=0, base=FAKE + 10 ** 9)
+    noscale.v_scale = None
+    st = lib.nomas_kvcache_select_i8_codes(ctypes.byref(src), ok_idx, 2, 0, ctypes.byref(noscale),
+                                           None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+    st = lib.nomas_kvcache_select_i8_codes(ctypes.byref(src), ok_idx, 2, 1, ctypes.byref(win),
+                                           None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG  # a device list needs dev_err
+
+
+def test_int8_attention_validation(lib):
+    q, o = FAKE, FAKE + 10 ** 9
+    hist = nm._KVSpanI8(FAKE + 2 * 10 ** 9, FAKE + 3 * 10 ** 9, FAKE + 4 * 10 ** 9,
+                        FAKE + 4 * 10 ** 9 + 10 ** 6, 1000)
+    spans = (nm._KVSpan * 4)(*[nm._KVSpan(FAKE + (5 + i) * 10 ** 9, FAKE + (9 + i) * 10 ** 9, 64)
+                               for i in range(4)])
+    st = lib.nomas_segment_attention_i8(q, 300, None, spans, 1, o, None, 0.0, 16, 128, None,
+                                        None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG            # no history struct
+    st = lib.nomas_segment_attention_i8(q, 300, ctypes.byref(hist), spans, 4, o, None, 0.0, 16,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED            # the history + 4 spans: one too many
+    st = lib.nomas_segment_attention_i8(q, 300, ctypes.byref(hist), spans, 3, o, None, 0.0, 8,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_UNSUPPORTED            # heads
+    bad = nm._KVSpanI8(hist.k, hist.v, hist.k_scale + 4, hist.v_scale, 1000)
+    st = lib.nomas_segment_attention_i8(q, 300, ctypes.byref(bad), spans, 1, o, None, 0.0, 16,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG            # misaligned scales
+    over = nm._KVSpanI8(o + ROW * 10, hist.v, hist.k_scale, hist.v_scale, 1000)
+    st = lib.nomas_segment_attention_i8(q, 300, ctypes.byref(over), spans, 1, o, None, 0.0, 16,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG            # codes overlap the output
+    neg = nm._KVSpanI8(hist.k, hist.v, hist.k_scale, hist.v_scale, -1)
+    st = lib.nomas_segment_attention_i8(q, 300, ctypes.byref(neg), spans, 1, o, None, 0.0, 16,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_INVALID_ARG
+
+
 def test_sparse_attention_validation(lib):
     spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 10 ** 9, FAKE + 2 * 10 ** 9, 300))
     o, lists, counts, err = FAKE + 3 * 10 ** 9, FAKE + 4 * 10 ** 9, FAKE + 5 * 10 ** 9, FAKE + 6 * 10 ** 9
