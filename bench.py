@@ -46,8 +46,8 @@ def parse_args():
                                           "sweep"],
                    default="720p")
     p.add_argument("--int8", action="store_true",
-                   help="bounded workload with an INT8 history cache (quantising append, "
-                        "dequantising gather)")
+                   help="bounded workload with the history in INT8 (quantising append, gather of "
+                        "codes and scales, attention dequantising the history tiles in the kernel)")
     p.add_argument("--sparse", type=float, default=0.0,
                    help="block-sparse attention keeping this fraction of the video key tiles "
                         "(text tiles always kept); 0 = dense")
@@ -147,6 +147,12 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- workload --
+def _mark(ev, name: str, which: int) -> None:
+    """Records the start (0) or end (1) event of `name` if the step is timed."""
+    if ev is not None and name in ev:
+        ev[name][which].record()
+
+
 class LayerStep:
     """Device-resident buffers of one layer-step and the launches of a step."""
 
@@ -178,6 +184,8 @@ class LayerStep:
         else:
             self.frames = None
         self.launches_per_step = 3 if self.frames else 2
+        self.append_kernels = "rope_append_kernel<bf16> (fused RoPE + append)"
+        self.select_kernel = "select_kernel"
         self.sparse = None
         self.shards = 0
         self.kv_splits = 1
@@ -191,7 +199,6 @@ class LayerStep:
         self.part_o = torch.empty((n_shards, w.n_q, 16, 128), dtype=torch.bfloat16,
                                   device="cuda")
         self.part_lse = torch.empty((n_shards, 16, w.n_q), dtype=torch.float32, device="cuda")
-        self.merge_ev = []
         self.launches_per_step += n_shards  # n_shards attention launches + 1 merge, was 1
 
     def _shard_spans(self, spans):
@@ -234,20 +241,25 @@ class LayerStep:
         return self.sparse_flops if self.sparse is not None else self.w.attention_flops()
 
     def run(self, ev=None, bufs=None):
+        """One layer-step; `ev` (optional) maps "append", "select" and "attn" to
+        (start, end) CUDA events recorded around those launches."""
         nm, w = self.nm, self.w
         ns = w.n_seg
         q, k, v, o = (self.q, self.k, self.v, self.o) if bufs is None else bufs
         self.cache.len = w.n_cache
+        _mark(ev, "append", 0)
         nm.kvcache_append(self.cache, k[:ns], v[:ns], q_in=q, q_out=self.q_rot,
                           layout=self.layout, cfg=self.cfg)
+        _mark(ev, "append", 1)
         if self.frames is not None:
+            _mark(ev, "select", 0)
             nm.kvcache_select(self.cache, self.frames, self.window)
+            _mark(ev, "select", 1)
             hist = self.window.span()
         else:
             hist = self.cache.span(0, w.n_cache)
         spans = [hist, (k[ns:], v[ns:]), self.cache.span(w.n_cache, w.n_cache + ns)]
-        if ev is not None:
-            ev[0].record()
+        _mark(ev, "attn", 0)
         if self.sparse is not None:
             nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=o, lse=self.lse,
                                         dev_err=self.err)
@@ -255,27 +267,23 @@ class LayerStep:
             for r, sub in enumerate(self._shard_spans(spans)):
                 nm.segment_attention(self.q_rot, sub, o=self.part_o[r],
                                      lse=self.part_lse[r].view(-1), dev_err=self.err)
-            if ev is not None:
-                mev = (self.torch.cuda.Event(enable_timing=True),
-                       self.torch.cuda.Event(enable_timing=True))
-                mev[0].record()
+            _mark(ev, "merge", 0)
             nm.attention_merge(self.part_o, self.part_lse, o=o, lse=self.lse)
-            if ev is not None:
-                mev[1].record()
-                self.merge_ev.append(mev)
+            _mark(ev, "merge", 1)
         else:
             nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err,
                                  kv_splits=self.kv_splits)
-        if ev is not None:
-            ev[1].record()
+        _mark(ev, "attn", 1)
 
 
 class LayerStepI8:
-    """Bounded-history layer-step with an INT8 history cache.
+    """Bounded-history layer-step with the history held in INT8 on the GPU.
 
     Per step: 3D RoPE of the segment's Q and K into bf16 buffers, the rotated
-    K and V quantised into the INT8 cache, the frame list gathered back to a
-    bf16 window, then attention over window + text + segment.
+    K and V quantised into the INT8 cache, the frame list gathered as codes
+    and scales into an INT8 window (4,224 B per token), then attention over
+    window + text + segment, the window's tiles dequantised inside the
+    attention kernel.
     """
 
     def __init__(self, wname: str, seed: int):
@@ -308,8 +316,11 @@ class LayerStepI8:
         self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.frames = bounded_frame_list(w, seed).tolist()
-        self.window = nm.KVCache.empty(w.n_window, 0)
-        self.launches_per_step = 4
+        self.window = nm.KVCacheI8.empty(w.n_window, 0)
+        # rope3d_qk, INT8 append, gather (codes, scales), attention
+        self.launches_per_step = 5
+        self.append_kernels = "rope_append_kernel<bf16> (RoPE of Q, K) + rope_append_kernel<int8>"
+        self.select_kernel = "select_kernel (codes, then scales)"
 
     def flops(self) -> float:
         return self.w.attention_flops()
@@ -319,15 +330,17 @@ class LayerStepI8:
         ns = w.n_seg
         q, k, v, o = (self.q, self.k, self.v, self.o) if bufs is None else bufs
         self.cache.len = w.n_cache
+        _mark(ev, "append", 0)
         nm.rope3d_qk(q, k, self.q_rot, self.k_rot, self.layout, self.cfg)
         nm.kvcache_append_i8(self.cache, self.k_rot[:ns], v[:ns])
+        _mark(ev, "append", 1)
+        _mark(ev, "select", 0)
         nm.kvcache_select(self.cache, self.frames, self.window)
+        _mark(ev, "select", 1)
         spans = [self.window.span(), (self.k_rot[ns:], v[ns:]), (self.k_rot[:ns], v[:ns])]
-        if ev is not None:
-            ev[0].record()
+        _mark(ev, "attn", 0)
         nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
-        if ev is not None:
-            ev[1].record()
+        _mark(ev, "attn", 1)
 
 
 class SweepStep:
@@ -339,7 +352,7 @@ class SweepStep:
     bf16 buffers, then attention over cache + text + segment.
     """
 
-    def __init__(self, seed: int):
+    def __init__(self, seed: int, layers: int | None = None):
         import torch
 
         import kv_cached_segment_b200 as nm
@@ -349,46 +362,62 @@ class SweepStep:
         w = self.w = WORKLOADS["720p"]
         dev = "cuda"
         ns, nt = w.n_seg, w.n_text
-        self.layers, self.steps_per_segment = SWEEP_LAYERS, SWEEP_STEPS
-        self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.seed = seed
+        self.layers = SWEEP_LAYERS if layers is None else layers
+        self.steps_per_segment = SWEEP_STEPS
         self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        # text rows of Q are copied by the RoPE pass; text K/V live with each layer
+        self.lay_q = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.lay_k = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, 0)
         self.cache = []
         for l in range(self.layers):
-            k = randn_bf16((w.n_cache + nt, 16, 128), seed * 1000 + 2 * l, dev)
-            v = randn_bf16((w.n_cache + nt, 16, 128), seed * 1000 + 2 * l + 1, dev)
+            k = randn_bf16((w.n_cache + nt, 16, 128), self.cache_seed(l, 0), dev)
+            v = randn_bf16((w.n_cache + nt, 16, 128), self.cache_seed(l, 1), dev)
             self.cache.append((k, v))
         self.inputs = [tuple(randn_bf16((w.n_q if i == 0 else ns, 16, 128),
-                                        seed * 100000 + 3 * s + i, dev) for i in range(3))
+                                        self.input_seed(s, i), dev) for i in range(3))
                        for s in range(self.steps_per_segment)]
         self.q_rot = torch.empty((w.n_q, 16, 128), dtype=torch.bfloat16, device=dev)
         self.k_rot = torch.empty((ns, 16, 128), dtype=torch.bfloat16, device=dev)
         self.o = torch.empty_like(self.q_rot)
+        self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.i = 0
         self.launches_per_step = 3 * self.layers
 
+    def cache_seed(self, layer: int, which: int) -> int:
+        """Seed of layer `layer`'s resident K (which 0) or V (1), text rows last."""
+        return self.seed * 1000 + 2 * layer + which
+
+    def input_seed(self, step: int, which: int) -> int:
+        """Seed of denoising step `step`'s Q (which 0), segment K (1), V (2)."""
+        return self.seed * 100000 + 3 * step + which
+
     def flops(self) -> float:
         return self.w.attention_flops() * self.layers
 
+    def spans(self, layer: int, v):
+        """Key/value spans of one layer: its cached rows, the text rows stored
+        with it, then the segment's rotated K (in k_rot) and its V."""
+        w = self.w
+        ck, cv = self.cache[layer]
+        return [(ck[:w.n_cache], cv[:w.n_cache]), (ck[w.n_cache:], cv[w.n_cache:]),
+                (self.k_rot, v)]
+
+    def run_layer(self, layer: int, q, k, v, lse=None):
+        nm = self.nm
+        nm.rope3d_qk(q, None, self.q_rot, None, self.lay_q, self.cfg)
+        nm.rope3d_qk(k, None, self.k_rot, None, self.lay_k, self.cfg)
+        nm.segment_attention(self.q_rot, self.spans(layer, v), o=self.o, lse=lse,
+                             dev_err=self.err)
+
     def run(self, ev=None):
-        nm, w = self.nm, self.w
-        ns, nt = w.n_seg, w.n_text
         q, k, v = self.inputs[self.i % self.steps_per_segment]
         self.i += 1
-        # text rows of Q are copied by the RoPE pass; text K/V live with each layer
-        lay_q = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
-        lay_k = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, 0)
-        if ev is not None:
-            ev[0].record()
-        for l in range(self.layers):
-            ck, cv = self.cache[l]
-            nm.rope3d_qk(q, None, self.q_rot, None, lay_q, self.cfg)
-            nm.rope3d_qk(k, None, self.k_rot, None, lay_k, self.cfg)
-            spans = [(ck[:w.n_cache], cv[:w.n_cache]), (ck[w.n_cache:], cv[w.n_cache:]),
-                     (self.k_rot, v)]
-            nm.segment_attention(self.q_rot, spans, o=self.o, dev_err=self.err)
-        if ev is not None:
-            ev[1].record()
+        _mark(ev, "attn", 0)
+        for layer in range(self.layers):
+            self.run_layer(layer, q, k, v)
+        _mark(ev, "attn", 1)
 
 
 def max_over_ranks(values, world: int, device):
@@ -401,6 +430,59 @@ def max_over_ranks(values, world: int, device):
     t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.tolist()]
+
+
+def rotated_query_rows(oracle, q_rows, rows, n_video: int, t, h, ww, split=(32, 48, 48),
+                       theta: float = 10000.0):
+    """The oracle's RoPE of sampled query rows (sorted, so video rows come
+    first); text rows (index >= n_video) pass unrotated."""
+    nv = int(np.count_nonzero(rows < n_video))
+    vid = rows[:nv]
+    return oracle.rope3d(q_rows, nv, t[vid], h[vid], ww[vid], split=split, theta=theta)
+
+
+def parity_summary(err_o, err_l, rows: int) -> dict:
+    parity = {"rows": rows, "max_abs_o": float(err_o.max()), "mean_abs_o": float(err_o.mean()),
+              "max_abs_lse": float(err_l.max()), "bar_max_abs": 2e-2, "bar_mean_abs": 2e-3}
+    parity["pass"] = bool(parity["max_abs_o"] <= 2e-2 and parity["mean_abs_o"] <= 2e-3
+                          and parity["max_abs_lse"] <= 2e-2)
+    return parity
+
+
+def sweep_parity(step, layer: int, n_rows: int = 24) -> dict:
+    """Runs one layer of the sweep (denoising step 0's inputs) and compares
+    sampled query rows, the first and last text rows among them, with the
+    fp64 oracle over that layer's spans built from the seeded inputs."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    def f64(x):
+        b = x.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+        return oracle.bf16_bits_to_f64(b)
+
+    w = step.w
+    ns = w.n_seg
+    q, k, v = step.inputs[0]
+    step.run_layer(layer, q, k, v, lse=step.lse)
+    torch.cuda.synchronize()
+    # the oracle starts from host copies of the seeded inputs (the layer's
+    # resident cache with its text rows, the step's Q, K, V), never from a
+    # kernel's output
+    ck, cv = (f64(x) for x in step.cache[layer])
+    qh, kh, vh = f64(q), f64(k), f64(v)
+    t, h, ww = oracle.video_positions(w.frames, w.grid_h, w.grid_w, w.t0)
+    spans = [(ck[:w.n_cache], cv[:w.n_cache]), (ck[w.n_cache:], cv[w.n_cache:]),
+             (oracle.rope3d(kh, ns, t, h, ww), vh)]
+    rows = np.random.default_rng(layer).integers(0, w.n_q, n_rows)
+    rows = np.unique(np.concatenate([rows, [0, ns - 1, ns, w.n_q - 1]]))
+    o_ref, l_ref = oracle.attention(rotated_query_rows(oracle, qh[rows], rows, ns, t, h, ww), spans)
+    err_o = np.abs(f64(step.o[torch.as_tensor(rows)]) - o_ref)
+    lse = step.lse.view(16, w.n_q).cpu().numpy().astype(np.float64)[:, rows]
+    out = parity_summary(err_o, np.abs(lse - l_ref), int(rows.size))
+    out["layer"] = layer
+    return out
 
 
 def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
@@ -436,9 +518,12 @@ def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
     refs = []
     t0 = time.perf_counter()
     while elapsed < budget_s and done < max_rows:
-        rows = np.sort(rng.integers(0, ns, rows_per_chunk))
-        q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
-                               ww[rows])
+        # every query row, text rows included (the last n_text rows)
+        rows = np.sort(rng.integers(0, w.n_q, rows_per_chunk))
+        if not refs:
+            rows[0], rows[-1] = ns, w.n_q - 1  # first and last text rows
+            rows = np.sort(rows)
+        q_rows = rotated_query_rows(oracle, f64(q_all[torch.as_tensor(rows)]), rows, ns, t, h, ww)
         refs.append((rows, oracle.attention(q_rows, spans)))
         done += rows.size
         elapsed = time.perf_counter() - t0
@@ -448,10 +533,8 @@ def cpu_oracle_rate(step, budget_s: float, rows_per_chunk: int, max_rows: int):
                             for r, (o, _) in refs])
     lse_gpu = step.lse.view(16, w.n_q).cpu().numpy().astype(np.float64)
     err_l = np.concatenate([np.abs(lse_gpu[:, r] - lse).ravel() for r, (_, lse) in refs])
-    parity = {"rows": done, "max_abs_o": float(err_o.max()), "mean_abs_o": float(err_o.mean()),
-              "max_abs_lse": float(err_l.max()), "bar_max_abs": 2e-2, "bar_mean_abs": 2e-3}
-    parity["pass"] = bool(parity["max_abs_o"] <= 2e-2 and parity["mean_abs_o"] <= 2e-3
-                          and parity["max_abs_lse"] <= 2e-2)
+    parity = parity_summary(err_o, err_l, done)
+    parity["text_rows"] = int(sum(np.count_nonzero(r >= ns) for r, _ in refs))
     return flops / elapsed / 1e12, done, elapsed, blas_threads(), parity
 
 
@@ -510,7 +593,7 @@ def workload_text(args, step) -> str:
                 f"({w.frames}x{w.grid_h}x{w.grid_w} segment + {w.n_text} text over "
                 f"{w.n_cache} cached tokens per layer)")
     hist = w.n_window if w.select_frames else w.n_cache
-    extra = " (INT8 history cache)" if args.int8 else ""
+    extra = " (history in INT8, dequantised in the attention kernel)" if args.int8 else ""
     if getattr(step, "kv_splits", 1) > 1:
         extra += f" (keys split {step.kv_splits} ways per query block, partials merged)"
     if getattr(args, "key_shards", 0) > 0:
@@ -565,9 +648,12 @@ def main():
     sampler = ClockSampler(uuid) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    def ev_pair():
+        return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    timed = step_kernels(step)
+    evs = [{name: ev_pair() for name in timed} for _ in range(args.steps)]
+    start, stop = ev_pair()
     barrier()
     torch.cuda.synchronize()
     start.record()
@@ -580,18 +666,40 @@ def main():
     if int(step.err.item()) != 0:
         raise RuntimeError(f"device error word {int(step.err.item())}")
 
-    merge_ms = 0.0
-    n_shards = getattr(step, "shards", 0)
-    if n_shards:
-        merge_ms = statistics.mean(a.elapsed_time(b) for a, b in step.merge_ev[:args.steps])
-    ms, attn_ms, merge_ms = max_over_ranks(
-        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for a, b in evs), merge_ms],
-        world, "cuda")
+    def mean_ms(name):
+        if name not in timed:
+            return 0.0
+        return statistics.mean(e[name][0].elapsed_time(e[name][1]) for e in evs)
+
+    ms, attn_ms, merge_ms, append_ms, select_ms = max_over_ranks(
+        [start.elapsed_time(stop), mean_ms("attn"), mean_ms("merge"), mean_ms("append"),
+         mean_ms("select")], world, "cuda")
     attn_ms -= merge_ms  # attention launches only
     ms_per_step = ms / args.steps
     flops = step.flops()
     value = flops * args.steps * world / (ms / 1e3) / 1e12
     attn_tflops = flops / (attn_ms / 1e3) / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+
+    # The memory-bound kernels against the copy bandwidth: the append (or
+    # RoPE + INT8 append) timed inside the steps above; the frame gather
+    # inside the steps when the workload has one, else a gather of every
+    # cached frame timed here on its own.
+    roof_append = roof_select = None
+    if "append" in timed:
+        a_bytes = append_bytes(step)
+        roof_append = memory_roofline(step.append_kernels, a_bytes, append_ms, hbm, peak_src,
+                                      "inside the timed steps")
+    if "select" in timed:
+        roof_select = memory_roofline(step.select_kernel, select_bytes(step, step.w.n_window),
+                                      select_ms, hbm, peak_src, "inside the timed steps")
+    elif isinstance(step, LayerStep):
+        sel_ms, n_tok = time_full_gather(step, repeats=20)
+        (sel_ms,) = max_over_ranks([sel_ms], world, "cuda")
+        roof_select = memory_roofline("select_kernel", select_bytes(step, n_tok), sel_ms, hbm,
+                                      peak_src, f"gather of all {n_tok // step.w.tokens_per_frame} "
+                                      f"cached frames ({n_tok} tokens) in a seeded order, mean "
+                                      f"of 20 launches timed alone")
 
     # ---- end to end through the public API with host buffers: every step
     # copies its inputs from pinned host memory and reads its output back;
@@ -617,10 +725,12 @@ def main():
         rate, rows, secs, threads, parity = cpu_oracle_rate(step, budget_s=12.0,
                                                             rows_per_chunk=16, max_rows=512)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "host": cpu_model(),
-               "sample": f"fp64 oracle RoPE + attention of {rows} sampled segment query rows "
-                         f"x 16 heads over all {step.w.n_k} keys ({secs:.1f} s)"}
+               "sample": f"fp64 oracle RoPE + attention of {rows} sampled query rows (segment "
+                         f"and text) x 16 heads over all {step.w.n_k} keys ({secs:.1f} s)"}
         if step.sparse is not None:
             parity = None  # the oracle above is dense attention
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "sweep":
+        parity = [sweep_parity(step, 0), sweep_parity(step, step.layers - 1)]
 
     if world > 1:
         dist.destroy_process_group()
@@ -638,18 +748,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {
-            "workload": workload_text(args, step),
-            "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
-            "attention_flops_per_step": flops,
-            "step": ("per layer: rope3d_qk x2 + segment attention" if args.workload == "sweep"
-                     else "rope3d_qk + int8 append + int8 select + segment attention" if args.int8
-                     else "fused rope3d+append" + (" + select" if w.select_frames else "")
-                     + " + segment attention"),
-            "l2": "inputs larger than L2: each step reads "
-                  f"{attn_per_step * (w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
-            "parallelism": f"independent layer-step per GPU x{world}",
-        },
+        "config": workload_config(args, step, world),
         # per GPU: value is the whole job's aggregate over `world` GPUs
         "pct_of_measured_bf16_peak": 100.0 * value / world / peak,
         "pct_of_datasheet_bf16_peak": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
@@ -658,23 +757,108 @@ def main():
                      "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 {peak_kind}",
                      "traffic": recorded_traffic(args.workload)},
+        "roofline_append": roof_append, "roofline_select": roof_select,
         "cpu_baseline": cpu, "e2e": e2e, "parity": parity,
         "gpu_launches": step.launches_per_step * args.steps * world,  # all ranks
         "clocks": clocks,
     }
+    n_shards = getattr(step, "shards", 0)
     if n_shards:
         # merge: R partial O rows (+ LSE) read, one O row (+ LSE) written per query row
         mbytes = (n_shards + 1) * w.n_q * (16 * 128 * 2 + 16 * 4)
-        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        out["config"]["key_shards"] = n_shards
-        out["merge"] = {"kernel": "merge_kernel", "bound": "hbm", "ms": merge_ms,
-                        "bytes": mbytes, "achieved": mbytes / (merge_ms / 1e3) / 1e9,
-                        "peak": hbm, "unit": "GB/s",
-                        "frac": mbytes / (merge_ms / 1e3) / 1e9 / hbm}
+        out["merge"] = memory_roofline("merge_kernel", mbytes, merge_ms, hbm, peak_src,
+                                       "inside the timed steps")
     if args.workload == "sweep":
         out["ms_per_segment"] = ms_per_step * step.steps_per_segment
         out["roofline"]["note"] = "per-step average over the 54 layers (rope3d_qk launches included)"
     print(json.dumps(out), flush=True)
+
+
+def step_kernels(step) -> list:
+    """Names of the launch groups a step records events around."""
+    if isinstance(step, SweepStep):
+        return ["attn"]
+    names = ["append", "attn"]
+    if getattr(step, "frames", None) is not None:
+        names.append("select")
+    if getattr(step, "shards", 0):
+        names.append("merge")
+    return names
+
+
+def append_bytes(step) -> float:
+    """Algorithmic HBM bytes of a step's append group.
+
+    Fused RoPE + append: 24 KiB per video token (Q, K, V read; Q', K', V
+    written) + 8 KiB per text row of Q (read and written).  INT8 path:
+    RoPE of every Q and K row (16 KiB per row), then the quantising append of
+    the video rows (K', V read: 8 KiB; codes + scales written: 4,224 B)."""
+    w = step.w
+    if isinstance(step, LayerStepI8):
+        return float(w.n_q * 16384 + w.n_seg * (8192 + 4224))
+    return float(w.n_seg * 24576 + w.n_text * 8192)
+
+
+def select_bytes(step, n_tokens: int) -> float:
+    """Frame gather: 16 KiB per token (K and V rows read and written); from
+    an INT8 cache into an INT8 window, 4,224 B read and written per token
+    (codes and scales of K and V)."""
+    if isinstance(step, LayerStepI8):
+        return float(n_tokens * 2 * 4224)
+    return float(n_tokens * 16384)
+
+
+def memory_roofline(kernel: str, nbytes: float, ms: float, hbm: float, peak_src: str,
+                    how: str) -> dict:
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": kernel, "bound": "hbm", "bytes": nbytes, "ms": ms, "achieved": achieved,
+            "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "peak_source": f"{peak_src} copy bandwidth", "timed": how}
+
+
+def time_full_gather(step, repeats: int):
+    """Mean time of gathering every cached frame (seeded order) into a window."""
+    import torch
+
+    w = step.w
+    frames = np.random.default_rng(11).permutation(w.cache_frames).astype(np.int32).tolist()
+    window = step.nm.KVCache.empty(w.n_cache, 0)
+    step.cache.len = w.n_cache
+    for _ in range(3):
+        step.nm.kvcache_select(step.cache, frames, window)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(repeats)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record()
+        step.nm.kvcache_select(step.cache, frames, window)
+        b.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    del window
+    return ms, w.n_cache
+
+
+def workload_config(args, step, world: int) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    w = step.w
+    attn_per_step = getattr(step, "layers", 1)
+    cfg = {
+        "workload": workload_text(args, step),
+        "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
+        "attention_flops_per_step": w.attention_flops() * attn_per_step,
+        "step": ("per layer: rope3d_qk x2 + segment attention" if args.workload == "sweep"
+                 else "rope3d_qk + int8 append + int8 select + segment attention over the "
+                      "int8 window" if args.int8
+                 else "fused rope3d+append" + (" + select" if w.select_frames else "")
+                 + " + segment attention"),
+        "l2": "inputs larger than L2: each step reads "
+              f"{attn_per_step * (w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
+        "parallelism": f"independent layer-step per GPU x{world}",
+    }
+    if getattr(args, "key_shards", 0):
+        cfg["key_shards"] = args.key_shards
+    return cfg
 
 
 class E2EPipeline:
@@ -771,9 +955,8 @@ def run_reference(args, rank, world):
     rng = np.random.default_rng(0)
 
     def one_step():
-        rows = np.sort(rng.integers(0, ns, rows_per_step))
-        q_rows = oracle.rope3d(f64(q_all[torch.as_tensor(rows)]), rows.size, t[rows], h[rows],
-                               ww[rows])
+        rows = np.sort(rng.integers(0, w.n_q, rows_per_step))  # segment and text rows
+        q_rows = rotated_query_rows(oracle, f64(q_all[torch.as_tensor(rows)]), rows, ns, t, h, ww)
         oracle.attention(q_rows, spans)
 
     for _ in range(max(3, args.warmup)):
@@ -794,20 +977,14 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": secs * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        # the same workload as the CUDA arm's line; what was sampled is in
-        # cpu_baseline.sample
-        "config": {"workload": workload_text(args, types.SimpleNamespace(w=w, kv_splits=1)),
-                   "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
-                   "attention_flops_per_step": w.attention_flops(),
-                   "step": "fused rope3d+append" + (" + select" if w.select_frames else "")
-                           + " + segment attention",
-                   "l2": "host memory (the oracle runs on the CPU)",
-                   "parallelism": "one process on the host cores"},
+        # the same workload and config as the CUDA arm's line; what this arm
+        # ran (host cores, a row sample) is in cpu_baseline
+        "config": workload_config(args, types.SimpleNamespace(w=w, kv_splits=1), world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "host": cpu_model(),
+                         "host": cpu_model(), "memory": "host memory, one process",
                          "sample": f"fp64 oracle RoPE + attention of {rows_per_step} sampled "
-                                   f"segment query rows per step x 16 heads over all {w.n_k} "
-                                   f"keys, {args.steps} steps"},
+                                   f"query rows (segment and text) per step x 16 heads over all "
+                                   f"{w.n_k} keys, {args.steps} steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
