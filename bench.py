@@ -11,7 +11,10 @@ over history + text + segment keys.  Prints ONE JSON line on rank 0.
   python bench.py --impl reference ...   # the fp64 CPU oracle, same metric
 
 Multi-GPU (torchrun): every rank runs its own independent layer-step (weak
-scaling, no collective on the data path); timing is the max over ranks.
+scaling, no collective on the data path); with --key-shards N on N GPUs the
+ranks instead share one layer-step, each attending over 1/N of the keys, the
+partials all-gathered over NCCL and merged (strong scaling).  Timing is the
+max over ranks.
 """
 from __future__ import annotations
 
@@ -53,8 +56,10 @@ def parse_args():
                         "(text tiles always kept); 0 = dense")
     p.add_argument("--key-shards", type=int, default=0,
                    help="split the key sequence into this many contiguous shards, attend over "
-                        "each into a partial (O, LSE) and merge them (the per-GPU work of "
-                        "key-sharded attention, on one GPU); 0 = one launch over all keys")
+                        "each into a partial (O, LSE) and merge them.  Equal to the number of "
+                        "GPUs: each rank holds one shard and the partials are all-gathered over "
+                        "NCCL; on one GPU with more shards: every shard on that GPU (the per-GPU "
+                        "work of key-sharded attention); 0 = one launch over all keys")
     p.add_argument("--kv-splits", default="1",
                    help="key splits of the attention launch (an integer, or 'auto': chosen from "
                         "the grid's wave count); 1 = one CTA per query block and head")
@@ -343,6 +348,109 @@ class LayerStepI8:
         _mark(ev, "attn", 1)
 
 
+def local_key_spans(span_lens, rank: int, world: int, align: int = 128):
+    """The rows of each key span that fall in this rank's contiguous share of
+    the concatenated key sequence (shares on `align`-key boundaries): a list
+    of (span index, first row, end row), in key order, empty spans left out."""
+    import kv_cached_segment_b200 as nm
+
+    a, b = nm.shard_rows(int(sum(span_lens)), rank, world, align=align)
+    out, base = [], 0
+    for s, n in enumerate(span_lens):
+        lo, hi = max(a, base), min(b, base + n)
+        if hi > lo:
+            out.append((s, lo - base, hi - base))
+        base += n
+    return out
+
+
+class ShardedLayerStep:
+    """A layer-step with its keys spread over the ranks (key-sharded attention,
+    as the pages' standard preset spreads the cache over eight GPUs).
+
+    Every rank holds a contiguous 1/N of the key sequence (history, then
+    text, then segment keys; shares on 128-key tiles) and all query rows.  Per
+    step each rank runs the fused RoPE + append of the segment (the rotated Q
+    and the segment's keys and values), attends with every query over its own
+    keys into a partial (O, LSE), all-gathers the partials over NCCL and
+    merges them (sharded_segment_attention).  The whole job computes one
+    layer-step: total work is fixed as N grows.
+    """
+
+    def __init__(self, wname: str, seed: int, rank: int, world: int):
+        import torch
+
+        import kv_cached_segment_b200 as nm
+        from seeded_inputs import WORKLOADS, randn_bf16
+
+        self.nm, self.torch = nm, torch
+        w = self.w = WORKLOADS[wname]
+        if w.select_frames:
+            raise SystemExit("key-sharded steps use a workload without a frame window")
+        dev = "cuda"
+        ns, nt = w.n_seg, w.n_text
+        self.rank, self.world = rank, world
+        self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
+        self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        # the same seeded inputs on every rank; each keeps only its share of
+        # the history
+        self.local = local_key_spans([w.n_cache, nt, ns], rank, world)
+        self.hist = None
+        for s, lo, hi in self.local:
+            if s == 0:
+                hk = randn_bf16((w.n_cache, 16, 128), seed * 16 + 4, dev)[lo:hi].clone()
+                hv = randn_bf16((w.n_cache, 16, 128), seed * 16 + 5, dev)[lo:hi].clone()
+                self.hist = (hk, hv)
+        torch.cuda.empty_cache()
+        self.seg = nm.KVCache.empty(ns, w.tokens_per_frame)
+        self.q = randn_bf16((w.n_q, 16, 128), seed * 16 + 1, dev)
+        self.k = randn_bf16((w.n_q, 16, 128), seed * 16 + 2, dev)
+        self.v = randn_bf16((w.n_q, 16, 128), seed * 16 + 3, dev)
+        self.q_rot = torch.empty_like(self.q)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.frames = None
+        # append, attention over the local share, two all-gathers (NCCL), merge
+        self.launches_per_step = 3
+        self.append_kernels = "rope_append_kernel<bf16> (fused RoPE + append)"
+        self.shards = world
+
+    def flops(self) -> float:
+        return self.w.attention_flops()  # of the whole job: every rank does 1/N
+
+    def local_flops(self) -> float:
+        keys = sum(hi - lo for _, lo, hi in self.local)
+        return 4.0 * self.w.n_q * keys * 128 * 16
+
+    def spans(self, k, v):
+        w, ns = self.w, self.w.n_seg
+        out = []
+        for s, lo, hi in self.local:
+            if s == 0:
+                out.append(self.hist)
+            elif s == 1:
+                out.append((k[ns + lo:ns + hi], v[ns + lo:ns + hi]))
+            else:
+                out.append(self.seg.span(lo, hi))
+        return out
+
+    def run(self, ev=None, bufs=None):
+        nm, w = self.nm, self.w
+        ns = w.n_seg
+        q, k, v, o = (self.q, self.k, self.v, self.o) if bufs is None else bufs
+        self.seg.len = 0
+        _mark(ev, "append", 0)
+        nm.kvcache_append(self.seg, k[:ns], v[:ns], q_in=q, q_out=self.q_rot, layout=self.layout,
+                          cfg=self.cfg)
+        _mark(ev, "append", 1)
+        _mark(ev, "attn", 0)
+        nm.sharded_segment_attention(
+            self.q_rot, self.spans(k, v), lse=self.lse,
+            merge=lambda op, lp, lse: nm.attention_merge(op, lp, o=o, lse=lse))
+        _mark(ev, "attn", 1)
+
+
 class SweepStep:
     """One denoising step of a whole segment: 54 layers of the 720p layer-step.
 
@@ -560,7 +668,14 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def make_step(args, rank):
+def make_step(args, rank, world=1):
+    if args.key_shards > 0 and args.key_shards == world:
+        if args.sparse > 0 or args.int8 or args.workload == "sweep" or args.kv_splits != "1":
+            raise SystemExit("--key-shards across ranks runs the dense bf16 layer-step only")
+        # one seed for all ranks: together they compute one layer-step
+        return ShardedLayerStep(args.workload, seed=1, rank=rank, world=world)
+    if args.key_shards > 0 and world > 1:
+        raise SystemExit("--key-shards across ranks must equal the number of GPUs")
     if args.workload == "sweep":
         return SweepStep(seed=1 + rank)
     if args.int8:
@@ -629,7 +744,8 @@ def main():
             dist.barrier()
 
     peaks, peak_src = load_peaks()
-    step = make_step(args, rank)
+    step = make_step(args, rank, world)
+    sharded = isinstance(step, ShardedLayerStep)
     torch.cuda.synchronize()
 
     warmup = max(3, args.warmup)
@@ -677,7 +793,10 @@ def main():
     attn_ms -= merge_ms  # attention launches only
     ms_per_step = ms / args.steps
     flops = step.flops()
-    value = flops * args.steps * world / (ms / 1e3) / 1e12
+    # replicas: every rank computes a layer-step; key shards: all ranks
+    # together compute one
+    jobs = 1 if sharded else world
+    value = flops * args.steps * jobs / (ms / 1e3) / 1e12
     attn_tflops = flops / (attn_ms / 1e3) / 1e12
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
 
@@ -693,7 +812,7 @@ def main():
     if "select" in timed:
         roof_select = memory_roofline(step.select_kernel, select_bytes(step, step.w.n_window),
                                       select_ms, hbm, peak_src, "inside the timed steps")
-    elif isinstance(step, LayerStep):
+    elif isinstance(step, (LayerStep, ShardedLayerStep)) and not sharded:
         sel_ms, n_tok = time_full_gather(step, repeats=20)
         (sel_ms,) = max_over_ranks([sel_ms], world, "cuda")
         roof_select = memory_roofline("select_kernel", select_bytes(step, n_tok), sel_ms, hbm,
@@ -706,7 +825,7 @@ def main():
     # two buffer sets and two copy streams overlap step i+1's upload and step
     # i-1's download with step i's kernels.
     e2e = None
-    if not args.no_e2e and args.workload != "sweep":
+    if not args.no_e2e and args.workload != "sweep" and not sharded:
         pipe = E2EPipeline(step)
         pipe.run(2)
         torch.cuda.synchronize()
@@ -747,7 +866,8 @@ def main():
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
         "config": workload_config(args, step, world),
         # per GPU: value is the whole job's aggregate over `world` GPUs
         "pct_of_measured_bf16_peak": 100.0 * value / world / peak,
@@ -763,7 +883,15 @@ def main():
         "clocks": clocks,
     }
     n_shards = getattr(step, "shards", 0)
-    if n_shards:
+    if sharded:
+        # attention_ms holds this rank's partial attention, the two
+        # all-gathers and the merge; the roofline counts this rank's keys
+        loc = step.local_flops()
+        out["roofline"].update({"achieved": loc / (attn_ms / 1e3) / 1e12,
+                                "frac": loc / (attn_ms / 1e3) / 1e12 / peak,
+                                "note": "per rank: partial attention over its key share + NCCL "
+                                        "all-gather of the partials + merge"})
+    elif n_shards:
         # merge: R partial O rows (+ LSE) read, one O row (+ LSE) written per query row
         mbytes = (n_shards + 1) * w.n_q * (16 * 128 * 2 + 16 * 4)
         out["merge"] = memory_roofline("merge_kernel", mbytes, merge_ms, hbm, peak_src,
@@ -778,6 +906,8 @@ def step_kernels(step) -> list:
     """Names of the launch groups a step records events around."""
     if isinstance(step, SweepStep):
         return ["attn"]
+    if isinstance(step, ShardedLayerStep):
+        return ["append", "attn"]
     names = ["append", "attn"]
     if getattr(step, "frames", None) is not None:
         names.append("select")
@@ -854,7 +984,9 @@ def workload_config(args, step, world: int) -> dict:
                  + " + segment attention"),
         "l2": "inputs larger than L2: each step reads "
               f"{attn_per_step * (w.n_q * 3 + w.n_k * 2) * 4096 / 1e9:.2f} GB > 126 MB",
-        "parallelism": f"independent layer-step per GPU x{world}",
+        "parallelism": (f"keys sharded over {world} GPUs (partials all-gathered over NCCL and "
+                        f"merged)" if isinstance(step, ShardedLayerStep)
+                        else f"independent layer-step per GPU x{world}"),
     }
     if getattr(args, "key_shards", 0):
         cfg["key_shards"] = args.key_shards

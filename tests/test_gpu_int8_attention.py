@@ -20,12 +20,15 @@ from tests._util import assert_close, bits, f64
 pytestmark = pytest.mark.gpu
 
 
-def _i8_history(n, seed, scale_max=0.05):
+def _i8_history(n, seed):
+    """Codes and scales shaped like a quantised N(0, 1) history: codes about
+    N(0, 40^2) clipped to +-127, scales near 1/40, so values are about
+    N(0, 1) like the bf16 spans; one (token, head) has scale 0."""
     g = torch.Generator().manual_seed(seed)
-    kc = torch.randint(-127, 128, (n, 16, 128), generator=g, dtype=torch.int8)
-    vc = torch.randint(-127, 128, (n, 16, 128), generator=g, dtype=torch.int8)
-    ks = torch.rand((n, 16), generator=g) * scale_max
-    vs = torch.rand((n, 16), generator=g) * scale_max
+    kc = (torch.randn((n, 16, 128), generator=g) * 40).round().clamp(-127, 127).to(torch.int8)
+    vc = (torch.randn((n, 16, 128), generator=g) * 40).round().clamp(-127, 127).to(torch.int8)
+    ks = (1.0 + 0.5 * torch.rand((n, 16), generator=g)) / 48.0
+    vs = (1.0 + 0.5 * torch.rand((n, 16), generator=g)) / 48.0
     if n > 3:
         ks[3, 5] = 0.0  # an all-zero (token, head)
         vs[3, 5] = 0.0

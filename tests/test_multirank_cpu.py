@@ -1,8 +1,11 @@
-"""Host logic of the multi-GPU bench on CPU: two gloo ranks.
+"""Host logic of the multi-GPU paths on CPU, with gloo ranks.
 
-bench.py runs one independent layer-step per rank (no collective on the data
-path) and reports the slowest rank's time; this checks that reduction with a
-world of two processes.
+bench.py either runs one independent layer-step per rank (no collective on
+the data path) or, with --key-shards equal to the number of GPUs, shares one
+layer-step over the ranks by keys (partials all-gathered and merged); it
+reports the slowest rank's time.  Checked here with two and three processes,
+the oracle standing in for the kernels: the cross-rank reduction, the
+binding's sharded attention, and the bench's split of the key sequence.
 """
 import os
 import socket
@@ -109,3 +112,79 @@ def test_shard_rows_covers_everything_once():
             cuts = [nm.shard_rows(n, r, world, align=920) for r in range(world)]
             assert cuts[0][0] == 0 and cuts[-1][1] == n
             assert all(cuts[i][1] == cuts[i + 1][0] for i in range(world - 1))
+
+
+def _bench_shard_worker(rank, world, port, out):
+    # The key-sharded bench step's orchestration, with the oracle standing in
+    # for the kernels: this rank's share of [history | text | segment] keys
+    # (bench.local_key_spans), partial attention, all-gather, merge.
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+
+    import bench
+    import kv_cached_segment_b200 as nm
+    import oracle
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(1)
+        lens = [700, 37, 300]  # history, text, segment; shares on 128-key tiles
+        q = torch.randn((23, 16, 128), generator=g, dtype=torch.float64)
+        kv = [(torch.randn((n, 16, 128), generator=g, dtype=torch.float64),
+               torch.randn((n, 16, 128), generator=g, dtype=torch.float64)) for n in lens]
+        local = bench.local_key_spans(lens, rank, world)
+        spans = [(kv[s][0][lo:hi], kv[s][1][lo:hi]) for s, lo, hi in local]
+
+        def attend(qq, sp, lse_out):
+            if not sp:
+                lse_out.fill_(-float("inf"))
+                return torch.zeros_like(qq)
+            o, l = oracle.attention(qq.numpy(), [(a.numpy(), b.numpy()) for a, b in sp])
+            lse_out.copy_(torch.from_numpy(l).reshape(-1))
+            return torch.from_numpy(o)
+
+        def merge(op, lp, lse_out):
+            o, _ = oracle.merge_partials(op.numpy(), lp.double().numpy())
+            return torch.from_numpy(o)
+
+        lse = torch.empty(16 * 23, dtype=torch.float32)
+        o = nm.sharded_segment_attention(q, spans, attend=attend, merge=merge, lse=lse)
+        o_ref, _ = oracle.attention(q.numpy(), [(a.numpy(), b.numpy()) for a, b in kv])
+        keys = sum(hi - lo for _, lo, hi in local)
+        out[rank] = (float(np.abs(o.numpy() - o_ref).max()), keys)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_key_shards_on_gloo_ranks():
+    for world in (2, 3):
+        ctx = mp.get_context("spawn")
+        mgr = ctx.Manager()
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_bench_shard_worker, args=(r, world, port, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=180)
+            assert p.exitcode == 0
+        assert all(out[r][0] < 1e-6 for r in range(world))
+        assert sum(out[r][1] for r in range(world)) == 700 + 37 + 300  # every key once
+
+
+def test_local_key_spans_partition_in_order():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    lens = [55200, 512, 27600]
+    for world in (1, 2, 3, 8):
+        seen = []
+        for r in range(world):
+            for s, lo, hi in bench.local_key_spans(lens, r, world):
+                base = sum(lens[:s])
+                seen.extend(range(base + lo, base + hi))
+        assert seen == list(range(sum(lens)))
