@@ -964,10 +964,10 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
     // converter warpgroups (warps 8-15) lower theirs at another, before the
     // roles diverge.
     if (warp < 8) {
-      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kI8SoftmaxRegs));
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kI8SoftmaxRegs) : "memory");
       role_softmax();
     } else {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kI8OtherRegs));
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kI8OtherRegs) : "memory");
       if (warp == kProducerWarp)
         role_producer();
       else if (warp == kMmaWarp)
