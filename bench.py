@@ -49,8 +49,9 @@ def parse_args():
                                           "sweep"],
                    default="720p")
     p.add_argument("--int8", action="store_true",
-                   help="bounded workload with the history in INT8 (quantising append, gather of "
-                        "codes and scales, attention dequantising the history tiles in the kernel)")
+                   help="the history in INT8 (quantising append; for a workload with a frame "
+                        "window, a gather of codes and scales; attention dequantising the "
+                        "history tiles in the kernel)")
     p.add_argument("--sparse", type=float, default=0.0,
                    help="block-sparse attention keeping this fraction of the video key tiles "
                         "(text tiles always kept); 0 = dense")
@@ -299,8 +300,6 @@ class LayerStepI8:
 
         self.nm, self.torch = nm, torch
         w = self.w = WORKLOADS[wname]
-        if not w.select_frames:
-            raise SystemExit("--int8 needs the bounded workload")
         dev = "cuda"
         ns, nt = w.n_seg, w.n_text
         self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
@@ -320,10 +319,12 @@ class LayerStepI8:
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(16 * w.n_q, dtype=torch.float32, device=dev)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.frames = bounded_frame_list(w, seed).tolist()
-        self.window = nm.KVCacheI8.empty(w.n_window, 0)
+        # with a frame window: the listed frames gathered as codes and scales;
+        # without one, attention reads the INT8 cache's history directly
+        self.frames = bounded_frame_list(w, seed).tolist() if w.select_frames else None
+        self.window = nm.KVCacheI8.empty(w.n_window, 0) if w.select_frames else None
         # rope3d_qk, INT8 append, gather (codes, scales), attention
-        self.launches_per_step = 5
+        self.launches_per_step = 5 if w.select_frames else 3
         self.append_kernels = "rope_append_kernel<bf16> (RoPE of Q, K) + rope_append_kernel<int8>"
         self.select_kernel = "select_kernel (codes, then scales)"
 
@@ -339,10 +340,14 @@ class LayerStepI8:
         nm.rope3d_qk(q, k, self.q_rot, self.k_rot, self.layout, self.cfg)
         nm.kvcache_append_i8(self.cache, self.k_rot[:ns], v[:ns])
         _mark(ev, "append", 1)
-        _mark(ev, "select", 0)
-        nm.kvcache_select(self.cache, self.frames, self.window)
-        _mark(ev, "select", 1)
-        spans = [self.window.span(), (self.k_rot[ns:], v[ns:]), (self.k_rot[:ns], v[:ns])]
+        if self.frames is not None:
+            _mark(ev, "select", 0)
+            nm.kvcache_select(self.cache, self.frames, self.window)
+            _mark(ev, "select", 1)
+            hist = self.window.span()
+        else:
+            hist = self.cache.span(0, w.n_cache)
+        spans = [hist, (self.k_rot[ns:], v[ns:]), (self.k_rot[:ns], v[:ns])]
         _mark(ev, "attn", 0)
         nm.segment_attention(self.q_rot, spans, o=o, lse=self.lse, dev_err=self.err)
         _mark(ev, "attn", 1)
@@ -978,8 +983,8 @@ def workload_config(args, step, world: int) -> dict:
         "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
         "attention_flops_per_step": w.attention_flops() * attn_per_step,
         "step": ("per layer: rope3d_qk x2 + segment attention" if args.workload == "sweep"
-                 else "rope3d_qk + int8 append + int8 select + segment attention over the "
-                      "int8 window" if args.int8
+                 else "rope3d_qk + int8 append + " + ("int8 select + " if w.select_frames else "")
+                      + "segment attention over the int8 history" if args.int8
                  else "fused rope3d+append" + (" + select" if w.select_frames else "")
                  + " + segment attention"),
         "l2": "inputs larger than L2: each step reads "

@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include "nomas_internal.h"
+#include "f32x2.cuh"
 
 namespace nomas {
 namespace {
@@ -57,8 +58,8 @@ __device__ __forceinline__ uint4 rot_chunk(uint4 v, const float (&c)[4], const f
 // transposed butterfly: at the first two xor steps a lane keeps half of its
 // items and trades the other half with its partner, so 2 + 1 + 1 + 1
 // shuffles leave lanes 4i..4i+3 holding item i reduced over the row.  Each
-// lane then does the divisions for its own item only, and 4 shuffles hand
-// every lane the reciprocal of each item.
+// lane then does the divisions for its own item only, and shuffles hand
+// every lane the reciprocals of each item.
 static_assert(kHeadGroup == 4, "the butterfly below reduces 4 items over 16 lanes");
 
 __device__ __forceinline__ float chunk_absmax(uint4 v) {
@@ -90,42 +91,48 @@ __device__ __forceinline__ float row_absmax_transposed(const float (&am)[kHeadGr
   return fmaxf(r, __shfl_xor_sync(row_mask, r, 1));
 }
 
-// 8 codes of one chunk.  Fast path: p = x * inv with inv = 127 / a, both
-// rounded to float32, is within 127 * 2^-23 < 2^-15 of the exact quotient
-// 127 x / a; adding 1.5 * 2^23 rounds p to an integer half to even and leaves
-// it, in two's complement, in the low byte of the sum (|p| < 127.5, so no
-// clamp is needed).  That integer is the exact quotient's nearest unless p
-// lies within 2^-15 of a half-integer.  There the value takes the exact path:
-// 127 x is exact in float32 and the correctly rounded quotient
-// fl(127 x / a) cannot sit on a half-integer unless the exact quotient does
-// (x and a carry 8 significant bits, so a quotient that is not a tie is more
-// than 2^-17 from one, above half a float32 step below 128), so rounding it
-// half to even gives the code (also used when a is so small that 127 / a
-// overflows).  The product is rounded to float32 before the
-// add: the scalar intrinsics below are never contracted into a fused
-// multiply-add.
+// 8 codes of one chunk.  Each value's quotient 127 x / a is formed in
+// float32 with one correction step: p = x * fl(127 / a) (within two units in
+// the last place), the residual r = 127 x - p a is exact in a fused
+// multiply-add, and q = p + r * fl(1 / a) is then within half a unit (plus
+// a negligible term) of the exact quotient: a faithful rounding of it.  A
+// quotient that is not itself a tie lies more than 2^-17 from one (x and a
+// carry 8 significant bits), more than a unit in the last place of any
+// quotient below 128, so both float32 neighbours of the exact quotient are on
+// its side of every half-integer, and an exact tie is representable and
+// returned exactly.  Rounding q to an integer half to even therefore gives
+// the code of the exact quotient.  That rounding is an add of 1.5 * 2^23,
+// which leaves the integer, in two's complement, in the low byte of the sum
+// (|q| < 127.5, so no clamp is needed).  When 127 / a overflows (a below
+// about 3.7e-37), the values take a correctly rounded division instead.
 __device__ __forceinline__ uint32_t round_magic(float x) {
   return __float_as_uint(__fadd_rn(x, 12582912.0f));  // 1.5 * 2^23
 }
-__device__ __forceinline__ uint2 quant_chunk(uint4 v, float inv, float amax) {
+__device__ __forceinline__ uint2 quant_chunk(uint4 v, float inv, float inv1, float amax) {
   constexpr float kMagic = 12582912.0f;
-  constexpr float kNearTie = 0.5f - 1.0f / 32768.0f;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float x[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
   uint32_t t[8];
+  if (inv <= 3.0e38f) {  // 127 / a finite (then 1 / a is too)
+    const uint64_t inv2 = f2(inv, inv), inv12 = f2(inv1, inv1), nega2 = f2(-amax, -amax);
+    const uint64_t c127 = f2(127.f, 127.f), magic2 = f2(kMagic, kMagic);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float p = __fmul_rn(x[i], inv);
-    t[i] = round_magic(p);
-    const float r = __fsub_rn(__uint_as_float(t[i]), kMagic);  // exact
-    // near a tie (exact difference), or 127 / a overflowed (a below ~3.7e-37)
-    if (fabsf(__fsub_rn(p, r)) >= kNearTie || !(fabsf(p) < 128.f))
-      t[i] = round_magic(__fdiv_rn(__fmul_rn(x[i], 127.f), amax));
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t xx = f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+      const uint64_t p = mul2(xx, inv2);
+      const uint64_t x127 = mul2(xx, c127);     // exact
+      const uint64_t r = fma2(p, nega2, x127);  // exact
+      const uint64_t q = fma2(r, inv12, p);
+      const float2 tv = unf2(add2(q, magic2));
+      t[2 * i] = __float_as_uint(tv.x);
+      t[2 * i + 1] = __float_as_uint(tv.y);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      t[2 * i] = round_magic(__fdiv_rn(__fmul_rn(__uint_as_float(w[i] << 16), 127.f), amax));
+      t[2 * i + 1] =
+          round_magic(__fdiv_rn(__fmul_rn(__uint_as_float(w[i] & 0xffff0000u), 127.f), amax));
+    }
   }
   const uint32_t lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040),
                                   0x5410);
@@ -225,6 +232,7 @@ rope_append_kernel(const __grid_constant__ RopeArgs a) {
         for (int g = 0; g < kHeadGroup; ++g) am[g] = chunk_absmax(src[g]);
         const float amax = row_absmax_transposed(am, cc, row_mask);
         const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+        const float inv1 = amax > 0.f ? __frcp_rn(amax) : 0.f;
         if ((cc & 3) == 0) scales[row * kHeads + h0 + (cc >> 2)] = __fdiv_rn(amax, 127.f);
 #pragma unroll
         for (int g = 0; g < kHeadGroup; ++g) {
@@ -232,8 +240,9 @@ rope_append_kernel(const __grid_constant__ RopeArgs a) {
           const int64_t coff = row * (kRowElems / 8) + (int64_t)(h0 + g) * 16 + cc;
           const int owner = (threadIdx.x & 16) + 4 * g;
           const float inv_g = __shfl_sync(row_mask, inv, owner);
+          const float inv1_g = __shfl_sync(row_mask, inv1, owner);
           const float amax_g = __shfl_sync(row_mask, amax, owner);
-          reinterpret_cast<uint2 *>(codes)[coff] = quant_chunk(src[g], inv_g, amax_g);
+          reinterpret_cast<uint2 *>(codes)[coff] = quant_chunk(src[g], inv_g, inv1_g, amax_g);
         }
       };
       if (do_k) {
