@@ -52,6 +52,10 @@ def parse_args():
                    help="the history in INT8 (quantising append; for a workload with a frame "
                         "window, a gather of codes and scales; attention dequantising the "
                         "history tiles in the kernel)")
+    p.add_argument("--int8-window", choices=["int8", "bf16"], default="int8",
+                   help="with --int8 and a frame window: keep the gathered window in INT8 and "
+                        "dequantise inside attention (int8), or dequantise once in the gather "
+                        "into a transient bf16 window read by the bf16 kernel (bf16)")
     p.add_argument("--sparse", type=float, default=0.0,
                    help="block-sparse attention keeping this fraction of the video key tiles "
                         "(text tiles always kept); 0 = dense")
@@ -292,7 +296,7 @@ class LayerStepI8:
     attention kernel.
     """
 
-    def __init__(self, wname: str, seed: int):
+    def __init__(self, wname: str, seed: int, window: str = "int8"):
         import torch
 
         import kv_cached_segment_b200 as nm
@@ -304,6 +308,7 @@ class LayerStepI8:
         ns, nt = w.n_seg, w.n_text
         self.layout = nm.SegLayout(w.frames, w.grid_h, w.grid_w, w.t0, nt)
         self.cfg = nm.RopeConfig(*w.rope_split, w.rope_theta)
+        self.window_kind = window if w.select_frames else "int8"
         self.cache = nm.KVCacheI8.empty(w.n_cache + ns, w.tokens_per_frame)
         chunk = 4 * w.tokens_per_frame * 30  # quantise the history in pieces
         for r0 in range(0, w.n_cache, chunk):
@@ -322,11 +327,17 @@ class LayerStepI8:
         # with a frame window: the listed frames gathered as codes and scales;
         # without one, attention reads the INT8 cache's history directly
         self.frames = bounded_frame_list(w, seed).tolist() if w.select_frames else None
-        self.window = nm.KVCacheI8.empty(w.n_window, 0) if w.select_frames else None
-        # rope3d_qk, INT8 append, gather (codes, scales), attention
-        self.launches_per_step = 5 if w.select_frames else 3
+        self.window = None
+        if w.select_frames:
+            self.window = (nm.KVCache.empty(w.n_window, 0) if self.window_kind == "bf16"
+                           else nm.KVCacheI8.empty(w.n_window, 0))
+        # rope3d_qk, INT8 append, gather (codes and scales: 2 launches; or one
+        # dequantising launch), attention
+        self.launches_per_step = 3 + (0 if not w.select_frames
+                                      else 1 if self.window_kind == "bf16" else 2)
         self.append_kernels = "rope_append_kernel<bf16> (RoPE of Q, K) + rope_append_kernel<int8>"
-        self.select_kernel = "select_kernel (codes, then scales)"
+        self.select_kernel = ("select_i8_kernel (gather + dequantise into bf16)"
+                              if self.window_kind == "bf16" else "select_kernel (codes, then scales)")
 
     def flops(self) -> float:
         return self.w.attention_flops()
@@ -684,7 +695,7 @@ def make_step(args, rank, world=1):
     if args.workload == "sweep":
         return SweepStep(seed=1 + rank)
     if args.int8:
-        return LayerStepI8(args.workload, seed=1 + rank)
+        return LayerStepI8(args.workload, seed=1 + rank, window=args.int8_window)
     step = LayerStep(args.workload, seed=1 + rank)
     if args.sparse > 0:
         step.use_sparse(args.sparse, seed=1 + rank)
@@ -713,7 +724,11 @@ def workload_text(args, step) -> str:
                 f"({w.frames}x{w.grid_h}x{w.grid_w} segment + {w.n_text} text over "
                 f"{w.n_cache} cached tokens per layer)")
     hist = w.n_window if w.select_frames else w.n_cache
-    extra = " (history in INT8, dequantised in the attention kernel)" if args.int8 else ""
+    extra = ""
+    if args.int8:
+        extra = (" (history in INT8; gathered frames dequantised once into a bf16 window)"
+                 if w.select_frames and getattr(args, "int8_window", "int8") == "bf16"
+                 else " (history in INT8, dequantised in the attention kernel)")
     if getattr(step, "kv_splits", 1) > 1:
         extra += f" (keys split {step.kv_splits} ways per query block, partials merged)"
     if getattr(args, "key_shards", 0) > 0:
@@ -937,8 +952,11 @@ def append_bytes(step) -> float:
 def select_bytes(step, n_tokens: int) -> float:
     """Frame gather: 16 KiB per token (K and V rows read and written); from
     an INT8 cache into an INT8 window, 4,224 B read and written per token
-    (codes and scales of K and V)."""
+    (codes and scales of K and V); dequantising into a bf16 window, 4,224 B
+    read and 8 KiB written."""
     if isinstance(step, LayerStepI8):
+        if step.window_kind == "bf16":
+            return float(n_tokens * (4224 + 8192))
         return float(n_tokens * 2 * 4224)
     return float(n_tokens * 16384)
 
@@ -983,8 +1001,12 @@ def workload_config(args, step, world: int) -> dict:
         "n_q": w.n_q, "n_k": w.n_k, "heads": 16, "head_dim": 128,
         "attention_flops_per_step": w.attention_flops() * attn_per_step,
         "step": ("per layer: rope3d_qk x2 + segment attention" if args.workload == "sweep"
-                 else "rope3d_qk + int8 append + " + ("int8 select + " if w.select_frames else "")
-                      + "segment attention over the int8 history" if args.int8
+                 else "rope3d_qk + int8 append + " + (
+                     ("dequantising select + segment attention over the bf16 window"
+                      if getattr(args, "int8_window", "int8") == "bf16" else
+                      "int8 select + segment attention over the int8 window")
+                     if w.select_frames else "segment attention over the int8 history")
+                 if args.int8
                  else "fused rope3d+append" + (" + select" if w.select_frames else "")
                  + " + segment attention"),
         "l2": "inputs larger than L2: each step reads "
