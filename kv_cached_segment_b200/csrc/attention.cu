@@ -394,10 +394,15 @@ __device__ __forceinline__ void convert_row(uint32_t src_row, uint32_t dst_row, 
                                             float scale) {
   const uint64_t sc2 = f2(scale, scale);
   const uint64_t off2 = f2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+  // All eight 16-byte loads of the row first: the shared-memory stores below
+  // would otherwise order each load after the previous chunk's stores and
+  // expose the load latency eight times.
+  uint32_t wq[8][4];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) lds128(src_row + (((uint32_t)q ^ sw) << 4), wq[q]);
 #pragma unroll
   for (int q = 0; q < 8; ++q) {  // 16 codes: dims 16q .. 16q + 15
-    uint32_t w[4];
-    lds128(src_row + (((uint32_t)q ^ sw) << 4), w);
+    const uint32_t(&w)[4] = wq[q];
     uint32_t out[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
