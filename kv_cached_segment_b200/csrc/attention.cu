@@ -40,6 +40,18 @@
 // Every wait is bounded (a globaltimer limit); on expiry the kernel records
 // NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, sets the
 // block's rows of O and LSE to NaN, frees TMEM and returns.
+//
+// INT8-history variant ("The 4090 preset": the resident frames stay on the
+// GPU in INT8; "Hy-Nomas en una RTX 4090", section "El preset de una GPU":
+// stored in INT8, computed in BF16): the first span holds INT8 codes and
+// per-(token, head) fp32 scales.  512 threads: warps 12-15 are a converter
+// warpgroup (warps 10-11 idle).  The producer TMA-loads each INT8 tile's
+// codes into one of two 16-KiB staging slots; converter thread r writes key
+// row r as bf16(code * scale) into the ring slot, in the layout a TMA load of
+// a bf16 tile gives, and one thread then arrives on the slot's full barrier,
+// so the MMA lane and the softmax run unchanged.  The ring has 4 slots here,
+// and setmaxnreg moves registers from the producer/MMA and converter
+// warpgroups to the softmax warpgroups.
 #include <atomic>
 
 #include <cuda_bf16.h>
