@@ -1,6 +1,6 @@
 """Fits the polynomial behind the FMA-pipe exp2 of the attention kernel.
 
-The kernel (csrc/attention.cu, ``exp2_poly_x2``) computes 2^x as 2^j * p(f)
+The kernel (csrc/attn_device.cuh, ``exp2_poly_x2``) computes 2^x as 2^j * p(f)
 with j = rint(x) and f = x - j in [-1/2, 1/2].  p is the degree-3 polynomial
 with the smallest maximum relative error to 2^f on that interval, found
 here by the Remez exchange algorithm; the kernel's constants kPc0..kPc3 are

@@ -15,7 +15,7 @@ import numpy as np
 from kv_cached_segment_b200.fit_exp2_poly import remez_exp2
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                   "kv_cached_segment_b200", "csrc", "attention.cu")
+                   "kv_cached_segment_b200", "csrc", "attn_device.cuh")
 
 
 def _constants():
