@@ -290,13 +290,49 @@ nomas_status nomas_temporal_context_frames(int32_t n_past, int32_t budget, float
  *                  usable.  The same holds in every attention entry point.
  *   testing_skip_kv_load: -1 in normal use.  For tests of the timeout path
  *                  only: a value k >= 0 makes every block leave out its k-th
- *                  K/V tile load (loads alternate K, V, K, V ... over the key
- *                  tiles), so a consumer wait cannot complete and must time out.
+ *                  K/V tile load (in the order its schedule loads them: K, V,
+ *                  K, V ... for TWO_TILE; K, K, K, then V, K, V, K ... for
+ *                  ONE_TILE and PAIR), so a consumer wait cannot complete and
+ *                  must time out.
+ *   pipeline:      the kernel schedule (NOMAS_ATTN_PIPELINE_*), 0 for the
+ *                  library default.
  */
 typedef struct {
   uint64_t wait_limit_ns;
   int32_t testing_skip_kv_load;
+  int32_t pipeline;  /* NOMAS_ATTN_PIPELINE_*; 0 = the library default */
 } nomas_attention_opts;
+
+/*
+ * Attention kernel schedules (same operation, arguments and results; they
+ * differ in speed only):
+ *   NOMAS_ATTN_PIPELINE_TWO_TILE: one CTA per 256 query rows as two 128-row
+ *     tiles that share each K/V tile, one score tile per query tile in TMEM.
+ *     The only schedule for block-sparse tile lists and INT8 histories.
+ *   NOMAS_ATTN_PIPELINE_ONE_TILE: one CTA per 128 query rows, three score
+ *     tiles in TMEM so that the scores of the next key tiles are computed
+ *     while the softmax works on the current one.
+ *   NOMAS_ATTN_PIPELINE_PAIR: as ONE_TILE, run by a cluster of two CTAs on two
+ *     SMs with 256-row tensor-core instructions (cta_group::2); each CTA
+ *     loads half of every K/V tile.
+ * Dense bf16 calls use NOMAS_ATTN_PIPELINE_DEFAULT_DENSE unless told
+ * otherwise (by their options or nomas_set_attention_pipeline); sparse and
+ * INT8 calls use TWO_TILE whatever the process default, and one that names
+ * ONE_TILE or PAIR in its options returns NOMAS_ERR_UNSUPPORTED.
+ */
+#define NOMAS_ATTN_PIPELINE_TWO_TILE 1
+#define NOMAS_ATTN_PIPELINE_ONE_TILE 2
+#define NOMAS_ATTN_PIPELINE_PAIR 3
+#define NOMAS_ATTN_PIPELINE_DEFAULT_DENSE NOMAS_ATTN_PIPELINE_TWO_TILE
+
+/*
+ * A setting of this library, with no counterpart on the pages: sets the
+ * schedule every later attention call of this process uses when its options
+ * name none (opts NULL or opts->pipeline 0), for dense bf16 calls; 0 restores
+ * the built-in choice.  Not synchronised with calls running on other host threads.
+ * Errors: NOMAS_ERR_INVALID_ARG for a value outside 0..3.
+ */
+nomas_status nomas_set_attention_pipeline(int32_t pipeline);
 
 /*
  * nomas_segment_attention ("How one segment is made": the joint attention of

@@ -53,6 +53,10 @@ NOMAS_ERR_CUDA = 5
 DEVERR_BAD_FRAME_INDEX = 0x1
 DEVERR_WAIT_TIMEOUT = 0x2
 MAX_SPANS = 4
+# Attention kernel schedules (NOMAS_ATTN_PIPELINE_* in nomas.h); 0 = default.
+PIPELINE_TWO_TILE = 1
+PIPELINE_ONE_TILE = 2
+PIPELINE_PAIR = 3
 MAX_MERGE_PARTS = 32
 MAX_MERGE_OUTPUTS = 32
 
@@ -75,6 +79,7 @@ EXPORTED_SYMBOLS = (
     "nomas_segment_attention_to_owners",
     "nomas_kvcache_select_i8_codes",
     "nomas_segment_attention_i8",
+    "nomas_set_attention_pipeline",
 )
 SPARSE_BLOCK_Q = 256
 SPARSE_BLOCK_K = 128
@@ -120,7 +125,8 @@ class _KVSpanI8(ctypes.Structure):
 
 
 class _AttnOpts(ctypes.Structure):
-    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("testing_skip_kv_load", ctypes.c_int32)]
+    _fields_ = [("wait_limit_ns", ctypes.c_uint64), ("testing_skip_kv_load", ctypes.c_int32),
+                ("pipeline", ctypes.c_int32)]
 
 
 _lib = None
@@ -185,6 +191,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.nomas_kvcache_select_i8_codes.restype = ctypes.c_int
     lib.nomas_kvcache_select_i8_codes.argtypes = [ctypes.POINTER(_KVCacheI8), P, I32, I32,
                                                   ctypes.POINTER(_KVCacheI8), P, P]
+    lib.nomas_set_attention_pipeline.restype = ctypes.c_int
+    lib.nomas_set_attention_pipeline.argtypes = [I32]
     lib.nomas_segment_attention_i8.restype = ctypes.c_int
     lib.nomas_segment_attention_i8.argtypes = [P, I64, ctypes.POINTER(_KVSpanI8),
                                                ctypes.POINTER(_KVSpan), I32, P, P, F32, I32, I32,
@@ -479,11 +487,13 @@ def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8
 
 def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, dev_err=None,
                       stream=None, wait_limit_ns: int = 0, testing_skip_kv_load: int = -1,
-                      kv_splits=1):
+                      kv_splits=1, pipeline: int = 0):
     """Attention of every row of q over all keys of ``spans`` (list of (k, v)); returns o.
 
     ``wait_limit_ns`` bounds every pipeline wait in the kernel (0: default);
     ``testing_skip_kv_load`` is for tests of the timeout path only.
+    ``pipeline`` picks the kernel schedule (``PIPELINE_*``; 0: the default,
+    see ``set_attention_pipeline``).
     ``kv_splits`` > 1 (or "auto", see ``auto_kv_splits``) cuts the key tiles
     into that many ranges computed by separate CTAs and merged, for shapes
     whose query blocks alone do not fill the GPU; the scratch for the
@@ -517,14 +527,15 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         kv_splits = auto_kv_splits(n_q, [int(k.shape[0]) for k, _ in spans], sm)
     kv_splits = int(kv_splits)
     if history is not None:
-        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load))
+        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load), int(pipeline))
         _check(lib.nomas_segment_attention_i8(_ptr(q), n_q, ctypes.byref(history), arr, len(spans),
                                               _ptr(o), _ptr(lse), float(softmax_scale), HEADS,
                                               HEAD_DIM, _ptr(dev_err), ctypes.byref(opts),
                                               _stream(stream)))
     elif kv_splits > 1:
-        if wait_limit_ns or testing_skip_kv_load != -1:
-            raise ValueError("kv_splits > 1 takes no wait_limit_ns / testing_skip_kv_load")
+        if wait_limit_ns or testing_skip_kv_load != -1 or pipeline:
+            raise ValueError("kv_splits > 1 takes no wait_limit_ns / testing_skip_kv_load / "
+                             "pipeline (set_attention_pipeline sets the default)")
         if stream is not None and not isinstance(stream, torch.cuda.Stream):
             raise TypeError("kv_splits > 1 takes stream=None or a torch.cuda.Stream")
         nbytes = lib.nomas_segment_attention_scratch_bytes(n_q, kv_splits)
@@ -537,8 +548,8 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         # one, the allocator must not hand the scratch out before they end
         if stream is not None:
             scratch.record_stream(stream)
-    elif wait_limit_ns or testing_skip_kv_load != -1:
-        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load))
+    elif wait_limit_ns or testing_skip_kv_load != -1 or pipeline:
+        opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load), int(pipeline))
         _check(lib.nomas_segment_attention_ex(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
                                               float(softmax_scale), HEADS, HEAD_DIM,
                                               _ptr(dev_err), ctypes.byref(opts), _stream(stream)))
@@ -547,6 +558,11 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
                                            float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
                                            _stream(stream)))
     return o
+
+
+def set_attention_pipeline(pipeline: int) -> None:
+    """Sets the schedule of later attention calls that name none (0: built-in)."""
+    _check(load_library().nomas_set_attention_pipeline(int(pipeline)))
 
 
 def segment_attention_sparse(q, spans, tile_list, tile_count, o=None, lse=None,

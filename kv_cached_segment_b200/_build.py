@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libnomas.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["abi.cu", "rope_append.cu", "select.cu", "attention.cu", "frame_picker.cu", "merge.cu",
+SOURCES = ["abi.cu", "rope_append.cu", "select.cu", "attention.cu", "attention_pair.cu", "frame_picker.cu", "merge.cu",
            "noalloc.cu"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -4,6 +4,7 @@
 // and kernel launches.  Every check happens before anything is launched, so a
 // rejected call leaves device memory untouched.  Nothing here allocates
 // device memory, synchronises or keeps a caller pointer past the call.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -130,13 +131,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D view of a [rows][16][128] bf16 tensor: inner extent 2048 elements, row
-// pitch 4096 B; box = 64 elements (128 B, one swizzle span) x 128 rows.
-nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows) {
+// pitch 4096 B; box = 64 elements (128 B, one swizzle span) x box_rows rows.
+nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows, uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {(cuuint64_t)kRowElems, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -339,6 +340,7 @@ nomas_status select_common(const CacheView &src, int32_t tokens_per_frame,
 }
 
 unsigned long long g_wait_limit_ns = 2000000000ull;  // 2 s per pipeline wait
+std::atomic<int32_t> g_pipeline{0};  // process default schedule, 0: built-in
 
 nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *spans,
                               int32_t n_spans, const int32_t *tile_list,
@@ -534,6 +536,13 @@ nomas_status nomas_kvcache_select_i8_codes(const nomas_kvcache_i8 *src, const in
   }
   window->tokens_per_frame = (int32_t)P;
   window->len = rows;
+  return ok();
+}
+
+nomas_status nomas_set_attention_pipeline(int32_t pipeline) {
+  if (pipeline < 0 || pipeline > NOMAS_ATTN_PIPELINE_PAIR)
+    return fail(NOMAS_ERR_INVALID_ARG, "unknown attention pipeline %d", pipeline);
+  g_pipeline.store(pipeline, std::memory_order_relaxed);
   return ok();
 }
 
@@ -734,6 +743,20 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   nomas_status st = check_shape(heads, head_dim);
   if (st != NOMAS_OK) return st;
   const bool i8 = i8_span != nullptr && i8_span->len != 0;
+  // Kernel schedule: the call's, else the process default, else the built-in
+  // choice; the one-tile and pair schedules take dense bf16 keys only.
+  // The process default applies to dense bf16 calls; a schedule named in the
+  // call's options must fit the call.
+  const bool dense_bf16 = !i8 && tile_list == nullptr;
+  int32_t pipeline = dense_bf16 ? g_pipeline.load(std::memory_order_relaxed) : 0;
+  if (opts != nullptr && opts->pipeline != 0) pipeline = opts->pipeline;
+  if (pipeline < 0 || pipeline > NOMAS_ATTN_PIPELINE_PAIR)
+    return fail(NOMAS_ERR_INVALID_ARG, "unknown attention pipeline %d", pipeline);
+  if (pipeline == 0) pipeline = dense_bf16 ? NOMAS_ATTN_PIPELINE_DEFAULT_DENSE : NOMAS_ATTN_PIPELINE_TWO_TILE;
+  if (pipeline != NOMAS_ATTN_PIPELINE_TWO_TILE && !dense_bf16)
+    return fail(NOMAS_ERR_UNSUPPORTED,
+                "the one-tile and pair attention schedules take dense bf16 keys only");
+  const uint32_t kv_box_rows = pipeline == NOMAS_ATTN_PIPELINE_PAIR ? 64u : 128u;
   if (i8_span != nullptr && (i8_span->len < 0 || i8_span->len > 0x7fff0000LL))
     return fail(NOMAS_ERR_INVALID_ARG, "INT8 history length out of range");
   if (i8 && (n_spans + 1 > kMaxSpans))
@@ -807,8 +830,8 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                             overlap(sp.v, sbytes, lse, n_q * kHeads * 4))) ||
         overlap(sp.k, sbytes, scratch, sb) || overlap(sp.v, sbytes, scratch, sb))
       return fail(NOMAS_ERR_INVALID_ARG, "span %d overlaps an output or the scratch", s);
-    if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len)) != NOMAS_OK) return st;
-    if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len)) != NOMAS_OK) return st;
+    if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len, kv_box_rows)) != NOMAS_OK) return st;
+    if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len, kv_box_rows)) != NOMAS_OK) return st;
     a.span_len[n_used] = sp.len;
     a.tile_base[n_used + 1] = a.tile_base[n_used] + (int32_t)((sp.len + 127) / 128);
     ++n_used;
@@ -872,7 +895,11 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
       return fail(NOMAS_ERR_INVALID_ARG, "testing_skip_kv_load must be >= -1");
     a.testing_skip_load = opts->testing_skip_kv_load;
   }
-  cudaError_t e = launch_attention(a, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      pipeline == NOMAS_ATTN_PIPELINE_TWO_TILE
+          ? launch_attention(a, static_cast<cudaStream_t>(stream))
+          : launch_attention_pair(a, pipeline == NOMAS_ATTN_PIPELINE_PAIR,
+                                  static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidKernelImage && a.i8)
     return fail(NOMAS_ERR_CUDA, "INT8 attention kernel not compiled to %d registers per thread at "
                 "launch; refusing to run its register split", 128);

@@ -113,6 +113,10 @@ struct AttnArgs {
   const float *i8_scale[2];
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
+// The one-tile (pair = false) and CTA-pair schedules: dense bf16 keys only,
+// K/V tensor maps with 128-row (one-tile) or 64-row (pair) boxes.
+bool attention_pair_supported(const AttnArgs &a);
+cudaError_t launch_attention_pair(const AttnArgs &a, bool pair, cudaStream_t stream);
 cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
                                    cudaStream_t stream);
 

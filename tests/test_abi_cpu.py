@@ -427,3 +427,32 @@ def test_every_entry_point_cites_its_passage():
         assert all(ln.startswith("#define") for ln in between), m.group(1)
         comment = before[start:end]
         assert '"' in comment or "no counterpart" in comment, m.group(1)
+
+
+def test_attention_pipeline_choice_validation(lib):
+    assert lib.nomas_set_attention_pipeline(4) == nm.NOMAS_ERR_INVALID_ARG
+    assert lib.nomas_set_attention_pipeline(-1) == nm.NOMAS_ERR_INVALID_ARG
+    for p in (nm.PIPELINE_TWO_TILE, nm.PIPELINE_ONE_TILE, nm.PIPELINE_PAIR, 0):
+        assert lib.nomas_set_attention_pipeline(p) == nm.NOMAS_OK
+    q, o = FAKE, FAKE + 10 ** 9
+    spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 2 * 10 ** 9, FAKE + 3 * 10 ** 9, 300))
+    for bad in (5, -2):
+        opts = nm._AttnOpts(0, -1, bad)
+        st = lib.nomas_segment_attention_ex(q, 100, spans, 1, o, None, 0.0, 16, 128, None,
+                                            ctypes.byref(opts), None)
+        assert st == nm.NOMAS_ERR_INVALID_ARG
+    # the one-tile and pair schedules take dense bf16 keys only
+    hist = nm._KVSpanI8(FAKE + 4 * 10 ** 9, FAKE + 5 * 10 ** 9, FAKE + 6 * 10 ** 9,
+                        FAKE + 6 * 10 ** 9 + 10 ** 6, 1000)
+    for p in (nm.PIPELINE_ONE_TILE, nm.PIPELINE_PAIR):
+        opts = nm._AttnOpts(0, -1, p)
+        st = lib.nomas_segment_attention_i8(q, 100, ctypes.byref(hist), spans, 1, o, None, 0.0, 16,
+                                            128, None, ctypes.byref(opts), None)
+        assert st == nm.NOMAS_ERR_UNSUPPORTED
+    # a process default of PAIR leaves INT8 calls on TWO_TILE: without a GPU
+    # driver the call gets past the schedule check and fails at the tensor map
+    assert lib.nomas_set_attention_pipeline(nm.PIPELINE_PAIR) == nm.NOMAS_OK
+    st = lib.nomas_segment_attention_i8(q, 100, ctypes.byref(hist), spans, 1, o, None, 0.0, 16,
+                                        128, None, None, None)
+    assert st == nm.NOMAS_ERR_CUDA, lib.nomas_last_error()
+    assert lib.nomas_set_attention_pipeline(0) == nm.NOMAS_OK

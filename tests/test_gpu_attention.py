@@ -13,6 +13,15 @@ from tests._util import assert_close, f64
 pytestmark = pytest.mark.gpu
 
 
+# Every test runs under each kernel schedule (same results expected).
+@pytest.fixture(autouse=True, params=[nm.PIPELINE_TWO_TILE, nm.PIPELINE_ONE_TILE, nm.PIPELINE_PAIR],
+                ids=["two_tile", "one_tile", "pair"])
+def pipeline(request):
+    nm.set_attention_pipeline(request.param)
+    yield request.param
+    nm.set_attention_pipeline(0)
+
+
 def _attn(q, spans, scale=0.0, want_lse=True):
     qd = q.cuda()
     sd = [(k.cuda(), v.cuda()) for k, v in spans]
