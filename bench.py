@@ -86,7 +86,7 @@ def kernel_source_hash() -> str:
     """Hash of the attention kernel's code: its sources with // comments and
     blank lines removed, so that editing a comment keeps a capture valid."""
     h = hashlib.sha256()
-    for name in ("attention.cu", "f32x2.cuh", "tmem_ops.cuh", "nomas_internal.h"):
+    for name in ("attention.cu", "attn_device.cuh", "f32x2.cuh", "tmem_ops.cuh", "nomas_internal.h"):
         with open(os.path.join(ROOT, "kv_cached_segment_b200", "csrc", name)) as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()

@@ -459,6 +459,11 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           const uint32_t acc = j > 0 ? 1u : 0u;
           const bool more = j + 1 < n_kv;
           if (!wait_phase(bar(kBarKVFull + slot_of(tv)), ph_of(tv), ctl)) break;
+          // The next K tile is waited for here, off the path from the P
+          // handoff to the next S (each wait costs ~100 cycles even when the
+          // phase is complete).  Its slot was freed by items consumed before
+          // this point, so the wait cannot hold up the ring.
+          if (more && !wait_phase(bar(kBarKVFull + slot_of(tk)), ph_of(tk), ctl)) break;
           if (!wait_phase(bar(kBarPHalf + 0), par, ctl)) break;
           tc_fence_after();
           issue_pv_half<0>(tO[0], tS[0], vd, acc);
@@ -466,8 +471,6 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           tc_fence_after();
           issue_pv_half<1>(tO[0], tS[0], vd, acc);
           if (more) {
-            if (!wait_phase(bar(kBarKVFull + slot_of(tk)), ph_of(tk), ctl)) break;
-            tc_fence_after();
             issue_qk(tS[0], dq0, kd);
             mma_commit(bar(kBarSFull + 0));
           } else {
