@@ -15,8 +15,9 @@
  *     and O rows have layout [tokens][heads][head_dim], contiguous; a row of
  *     16 x 128 bf16 is 4096 bytes.  Every tensor pointer must be 16-byte
  *     aligned.
- *   - Only heads = 16 and head_dim = 128 are implemented; other values return
- *     NOMAS_ERR_UNSUPPORTED.
+ *   - Only heads = 16 and head_dim = 128 are implemented (and 1, 2, 4 or 8
+ *     heads for nomas_segment_attention and nomas_segment_attention_ex on
+ *     dense bf16 spans); other values return NOMAS_ERR_UNSUPPORTED.
  *   - Every call is asynchronous on the caller's stream (`stream` is a
  *     cudaStream_t; NULL is the legacy default stream) and never synchronises.
  *     Argument errors are detected on the host before anything is launched and
@@ -43,7 +44,7 @@ typedef enum {
   NOMAS_ERR_INVALID_ARG = 1, /* NULL / misaligned pointer, bad size or layout */
   NOMAS_ERR_CAPACITY = 2,    /* a write would run past a cache's capacity     */
   NOMAS_ERR_INDEX = 3,       /* a host frame index outside the source cache   */
-  NOMAS_ERR_UNSUPPORTED = 4, /* heads != 16 or head_dim != 128, too many spans */
+  NOMAS_ERR_UNSUPPORTED = 4, /* a head count or head_dim not implemented, too many spans */
   NOMAS_ERR_CUDA = 5         /* a CUDA runtime/driver call failed             */
 } nomas_status;
 
@@ -191,6 +192,11 @@ nomas_status nomas_kvcache_select(const nomas_kvcache *src, const int32_t *frame
  *   lse    : optional fp32 [heads][n_q] output (natural log); NULL to skip.
  *   softmax_scale: <= 0 selects 1/sqrt(head_dim).
  *   dev_err: optional device int32 (see the conventions above).
+ *   heads  : 16; or 1, 2, 4 or 8 ("What 'world memory' stores": the cache
+ *            spread over 8 GPUs; with attention sharded by heads each GPU
+ *            holds all rows for its share of the heads), in which case q, the
+ *            spans and o hold that many heads per row and lse is
+ *            [heads][n_q].  head_dim: 128.
  * With no keys at all, O = 0 and LSE = -inf.  bf16 operands, fp32 scores,
  * softmax and accumulation; O rounded to bf16 to nearest-even.
  * Errors: NOMAS_ERR_INVALID_ARG, NOMAS_ERR_UNSUPPORTED, NOMAS_ERR_CUDA.

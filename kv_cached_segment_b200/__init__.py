@@ -22,7 +22,9 @@ Entry points (same names as the C ABI, without the ``nomas_`` prefix):
 Holders: ``KVCache`` and ``KVCacheI8`` (caller-owned device buffers plus
 ``len``), ``RopeConfig`` and ``SegLayout``.
 
-Key-sharded attention over several GPUs, in three forms:
+Head-sharded attention over several GPUs (``head_sharded_segment_attention``:
+all-to-all of the query and key rows by heads, attention over 16/world heads,
+all-to-all back).  Key-sharded attention over several GPUs, in three forms:
 ``sharded_segment_attention`` (partial attention per rank, NCCL all-gather of
 the partials, merge); ``peer_partial_attention`` + ``peer_merge_owned_rows``
 (the all-gather replaced by a merge that reads the owned rows of every GPU's
@@ -241,11 +243,11 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _rows(t: torch.Tensor, name: str) -> int:
+def _rows(t: torch.Tensor, name: str, heads: int = HEADS) -> int:
     if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
         raise TypeError(f"{name} must be a contiguous CUDA bf16 tensor")
-    if t.dim() != 3 or t.shape[1] != HEADS or t.shape[2] != HEAD_DIM:
-        raise ValueError(f"{name} must have shape [N][{HEADS}][{HEAD_DIM}], got {tuple(t.shape)}")
+    if t.dim() != 3 or t.shape[1] != heads or t.shape[2] != HEAD_DIM:
+        raise ValueError(f"{name} must have shape [N][{heads}][{HEAD_DIM}], got {tuple(t.shape)}")
     return t.shape[0]
 
 
@@ -500,12 +502,16 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
     partial results is allocated here, through PyTorch.
     """
     lib = load_library()
-    n_q = _rows(q, "q")
+    # Heads per row: 16, or 1, 2, 4 or 8 for a head-sharded dense call.
+    heads = int(q.shape[1]) if q.dim() == 3 else HEADS
+    if heads not in (1, 2, 4, 8, HEADS):
+        raise ValueError(f"q must have 16 heads (or 1, 2, 4 or 8), got {tuple(q.shape)}")
+    n_q = _rows(q, "q", heads)
     if o is None:
         o = torch.empty_like(q)
-    _rows(o, "o")
+    _rows(o, "o", heads)
     if lse is not None and (lse.dtype != torch.float32 or not lse.is_cuda or
-                            lse.numel() != HEADS * n_q or not lse.is_contiguous()):
+                            lse.numel() != heads * n_q or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous CUDA fp32 tensor of heads * n_q elements")
     if len(spans) > MAX_SPANS:
         raise ValueError(f"at most {MAX_SPANS} spans")
@@ -514,10 +520,14 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         history, spans = spans[0]._c(), list(spans[1:])
         if kv_splits not in (1, "1"):
             raise ValueError("an INT8 history span takes kv_splits=1")
+    if heads != HEADS and kv_splits == "auto":
+        kv_splits = 1
+    if heads != HEADS and (history is not None or kv_splits not in (1, "1")):
+        raise ValueError("fewer than 16 heads: dense bf16 spans and kv_splits=1 only")
     arr = (_KVSpan * max(1, len(spans)))()
     for i, (k, v) in enumerate(spans):
-        nk = _rows(k, f"span {i} k")
-        if _rows(v, f"span {i} v") != nk:
+        nk = _rows(k, f"span {i} k", heads)
+        if _rows(v, f"span {i} v", heads) != nk:
             raise ValueError(f"span {i}: k and v differ in rows")
         arr[i] = _KVSpan(k.data_ptr() if nk else None, v.data_ptr() if nk else None, nk)
     if dev_err is not None and (dev_err.dtype != torch.int32 or not dev_err.is_cuda):
@@ -551,11 +561,11 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
     elif wait_limit_ns or testing_skip_kv_load != -1 or pipeline:
         opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load), int(pipeline))
         _check(lib.nomas_segment_attention_ex(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
-                                              float(softmax_scale), HEADS, HEAD_DIM,
+                                              float(softmax_scale), heads, HEAD_DIM,
                                               _ptr(dev_err), ctypes.byref(opts), _stream(stream)))
     else:
         _check(lib.nomas_segment_attention(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
-                                           float(softmax_scale), HEADS, HEAD_DIM, _ptr(dev_err),
+                                           float(softmax_scale), heads, HEAD_DIM, _ptr(dev_err),
                                            _stream(stream)))
     return o
 
@@ -751,6 +761,87 @@ def peer_merge_owned_rows(part_o_peers, part_lse_peers, o_peers, lse_peers, rank
     n_q = part_o_peers[0].shape[0]
     a, b = shard_rows(n_q, rank, world, align=16)
     attention_merge_peers(part_o_peers, part_lse_peers, o_peers, lse_peers, row0=a, n_rows=b - a)
+
+
+def _all_to_all_rows(t, send_rows, recv_rows, group):
+    """all_to_all_single over dim 0 with per-rank row counts; bf16 moves as
+    int16 (a bit copy), so that backends without bf16 collectives work."""
+    import torch.distributed as dist
+
+    out = torch.empty((sum(recv_rows),) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+    a, b = (out.view(torch.int16), t.view(torch.int16)) if t.dtype == torch.bfloat16 else (out, t)
+    dist.all_to_all_single(a, b.contiguous(), output_split_sizes=list(recv_rows),
+                           input_split_sizes=list(send_rows), group=group)
+    return out
+
+
+def head_sharded_segment_attention(q, local_spans, group=None, lse=None, attend=None):
+    """Attention with the rows of Q and of the keys spread across the ranks of
+    `group` (sequence parallel), computed head-parallel (Ulysses-style): one
+    all-to-all gives every rank all query and key rows for 16/world of the
+    heads, each rank attends over those heads, and a second all-to-all
+    returns every rank its own query rows for all 16 heads.
+
+    q: this rank's query rows [n_q_local][16][128]; local_spans: this rank's
+    key/value rows (list of (k, v), [n][16][128]); the world size divides 16.
+    Returns O for the local query rows; fills lse ([16][n_q_local], fp32) if
+    given.  `attend(q_heads, spans, lse_heads)` defaults to segment_attention
+    (which takes 16/world heads per row)."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if HEADS % world:
+        raise ValueError(f"the world size must divide {HEADS} (got {world})")
+    hl = HEADS // world
+    attend = attend or (lambda qq, spans, l: segment_attention(qq, spans, lse=l))
+    n_q = q.shape[0]
+    dev = q.device
+    if local_spans:
+        k_loc = torch.cat([k for k, _ in local_spans]) if len(local_spans) > 1 else local_spans[0][0]
+        v_loc = torch.cat([v for _, v in local_spans]) if len(local_spans) > 1 else local_spans[0][1]
+    else:
+        k_loc = q.new_empty((0, HEADS, HEAD_DIM))
+        v_loc = q.new_empty((0, HEADS, HEAD_DIM))
+    n_k = k_loc.shape[0]
+    if world == 1:
+        rows_q, rows_k = [n_q], [n_k]
+    else:
+        cnt = torch.tensor([n_q, n_k], dtype=torch.int64,
+                           device=dev if dist.get_backend(group) == "nccl" else "cpu")
+        allc = [torch.empty_like(cnt) for _ in range(world)]
+        dist.all_gather(allc, cnt, group=group)
+        rows_q = [int(c[0]) for c in allc]
+        rows_k = [int(c[1]) for c in allc]
+
+    def to_heads(t, n_local, rows_all):
+        # [n][world][hl][128] -> per destination rank d, this rank's rows of
+        # heads d*hl .. d*hl + hl - 1; received in source-rank order.
+        send = t.reshape(n_local, world, hl, HEAD_DIM).transpose(0, 1).reshape(
+            world * n_local, hl, HEAD_DIM)
+        if world == 1:
+            return send.contiguous()
+        return _all_to_all_rows(send, [n_local] * world, rows_all, group)
+
+    q_h = to_heads(q, n_q, rows_q)
+    k_h = to_heads(k_loc, n_k, rows_k)
+    v_h = to_heads(v_loc, n_k, rows_k)
+    lse_h = torch.empty(hl * sum(rows_q), dtype=torch.float32, device=dev)
+    o_h = attend(q_h, [(k_h, v_h)] if k_h.shape[0] else [], lse_h)
+    # back: the rows of rank d (rows_q[d] of them, in order) to rank d
+    if world == 1:
+        o_back = o_h.reshape(1, n_q, hl, HEAD_DIM)
+    else:
+        o_back = _all_to_all_rows(o_h.contiguous(), rows_q, [n_q] * world, group).reshape(
+            world, n_q, hl, HEAD_DIM)
+    o = o_back.transpose(0, 1).reshape(n_q, HEADS, HEAD_DIM).contiguous()
+    if lse is not None:
+        lh = lse_h.view(hl, sum(rows_q)).t().contiguous()  # [rows][hl]
+        if world == 1:
+            lb = lh.reshape(1, n_q, hl)
+        else:
+            lb = _all_to_all_rows(lh, rows_q, [n_q] * world, group).reshape(world, n_q, hl)
+        lse.view(HEADS, n_q).copy_(lb.permute(0, 2, 1).reshape(HEADS, n_q))
+    return o
 
 
 def sharded_segment_attention(q, local_spans, group=None, lse=None, attend=None, merge=None):

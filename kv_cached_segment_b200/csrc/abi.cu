@@ -130,13 +130,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D view of a [rows][16][128] bf16 tensor: inner extent 2048 elements, row
-// pitch 4096 B; box = 64 elements (128 B, one swizzle span) x box_rows rows.
-nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows, uint32_t box_rows = 128) {
+// 2-D view of a [rows][heads][128] bf16 tensor (heads 16 unless a
+// head-sharded call has fewer): inner extent heads x 128 elements, row pitch
+// heads x 256 B; box = 64 elements (128 B, one swizzle span) x box_rows rows.
+nomas_status rows_map(CUtensorMap *m, const void *ptr, int64_t rows, uint32_t box_rows = 128,
+                      int32_t heads = kHeads) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return fail(NOMAS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t dims[2] = {(cuuint64_t)kRowElems, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+  const cuuint64_t dims[2] = {(cuuint64_t)heads * kHeadDim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)heads * kHeadDim * 2};
   const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims,
@@ -740,8 +742,18 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
                               const OwnerRouting *routing, void *stream,
                               const nomas_kv_span_i8 *i8_span) {
-  nomas_status st = check_shape(heads, head_dim);
-  if (st != NOMAS_OK) return st;
+  // Heads per row: 16, or for a dense bf16 call without key splits or routed
+  // outputs 1, 2, 4 or 8 (the local heads of a head-sharded layout).
+  const bool few_heads_ok = (i8_span == nullptr || i8_span->len == 0) && tile_list == nullptr &&
+                            kv_splits == 1 && routing == nullptr;
+  if (head_dim != kHeadDim ||
+      !(heads == kHeads || (few_heads_ok && (heads == 1 || heads == 2 || heads == 4 || heads == 8))))
+    return fail(NOMAS_ERR_UNSUPPORTED,
+                "heads=%d, head_dim=%d not implemented (16 heads of 128; 1, 2, 4 or 8 heads for "
+                "dense bf16 calls without key splits)", heads, head_dim);
+  nomas_status st = NOMAS_OK;
+  // Bytes of one row of Q, K, V or O, and of one query's LSE values.
+  const int64_t row_bytes = (int64_t)heads * kHeadDim * 2, lse_row = (int64_t)heads * 4;
   const bool i8 = i8_span != nullptr && i8_span->len != 0;
   // Kernel schedule: the call's, else the process default, else the built-in
   // choice; the one-tile and pair schedules take dense bf16 keys only.
@@ -776,9 +788,9 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return fail(NOMAS_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (!std::isfinite(softmax_scale)) return fail(NOMAS_ERR_INVALID_ARG, "softmax_scale not finite");
-  const int64_t qb = n_q * kRowBytes;
+  const int64_t qb = n_q * row_bytes;
   if (overlap(q, qb, o, qb)) return fail(NOMAS_ERR_INVALID_ARG, "o overlaps q");
-  if (lse != nullptr && (overlap(lse, n_q * kHeads * 4, o, qb) || overlap(lse, n_q * kHeads * 4, q, qb)))
+  if (lse != nullptr && (overlap(lse, n_q * lse_row, o, qb) || overlap(lse, n_q * lse_row, q, qb)))
     return fail(NOMAS_ERR_INVALID_ARG, "lse overlaps q or o");
   const int64_t sb = kv_splits > 1 ? split_scratch_bytes(n_q, kv_splits) : 0;
   if (kv_splits > 1) {
@@ -788,7 +800,7 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
       return fail(NOMAS_ERR_CAPACITY, "scratch of %lld bytes, %lld needed", (long long)scratch_bytes,
                   (long long)sb);
     if (overlap(scratch, sb, q, qb) || overlap(scratch, sb, o, qb) ||
-        (lse != nullptr && overlap(scratch, sb, lse, n_q * kHeads * 4)))
+        (lse != nullptr && overlap(scratch, sb, lse, n_q * lse_row)))
       return fail(NOMAS_ERR_INVALID_ARG, "scratch overlaps q, o or lse");
   }
   AttnArgs a{};
@@ -805,7 +817,7 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
     const int64_t sizes[4] = {cb, cb, scb, scb};
     for (int i = 0; i < 4; ++i)
       if (overlap(parts[i], sizes[i], o, qb) ||
-          (lse != nullptr && overlap(parts[i], sizes[i], lse, n_q * kHeads * 4)) ||
+          (lse != nullptr && overlap(parts[i], sizes[i], lse, n_q * lse_row)) ||
           overlap(parts[i], sizes[i], scratch, sb))
         return fail(NOMAS_ERR_INVALID_ARG, "INT8 history overlaps an output or the scratch");
     if ((st = codes_map(&a.tmap_k[0], h.k, h.len)) != NOMAS_OK) return st;
@@ -824,14 +836,14 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
     if (sp.len == 0) continue;
     if (sp.k == nullptr || sp.v == nullptr || !aligned16(sp.k) || !aligned16(sp.v))
       return fail(NOMAS_ERR_INVALID_ARG, "span %d k/v must be non-NULL and 16-byte aligned", s);
-    const int64_t sbytes = sp.len * kRowBytes;
+    const int64_t sbytes = sp.len * row_bytes;
     if (overlap(sp.k, sbytes, o, qb) || overlap(sp.v, sbytes, o, qb) ||
-        (lse != nullptr && (overlap(sp.k, sbytes, lse, n_q * kHeads * 4) ||
-                            overlap(sp.v, sbytes, lse, n_q * kHeads * 4))) ||
+        (lse != nullptr && (overlap(sp.k, sbytes, lse, n_q * lse_row) ||
+                            overlap(sp.v, sbytes, lse, n_q * lse_row))) ||
         overlap(sp.k, sbytes, scratch, sb) || overlap(sp.v, sbytes, scratch, sb))
       return fail(NOMAS_ERR_INVALID_ARG, "span %d overlaps an output or the scratch", s);
-    if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len, kv_box_rows)) != NOMAS_OK) return st;
-    if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len, kv_box_rows)) != NOMAS_OK) return st;
+    if ((st = rows_map(&a.tmap_k[n_used], sp.k, sp.len, kv_box_rows, heads)) != NOMAS_OK) return st;
+    if ((st = rows_map(&a.tmap_v[n_used], sp.v, sp.len, kv_box_rows, heads)) != NOMAS_OK) return st;
     a.span_len[n_used] = sp.len;
     a.tile_base[n_used + 1] = a.tile_base[n_used] + (int32_t)((sp.len + 127) / 128);
     ++n_used;
@@ -845,18 +857,19 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
       for (int s = 0; s < routing->n_owners; ++s) {
         const cudaError_t e = launch_attention_empty(
             static_cast<uint16_t *>(routing->o[s]) + (int64_t)routing->slot * n_q * kRowElems,
-            routing->lse[s] + (int64_t)routing->slot * kHeads * n_q, n_q,
+            routing->lse[s] + (int64_t)routing->slot * kHeads * n_q, n_q, kHeads,
             static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "attention (no keys) launch");
       }
       return ok();
     }
-    const cudaError_t e = launch_attention_empty(static_cast<uint16_t *>(o), lse, n_q,
+    const cudaError_t e = launch_attention_empty(static_cast<uint16_t *>(o), lse, n_q, heads,
                                                  static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention (no keys) launch");
     return ok();
   }
-  if ((st = rows_map(&a.tmap_q, q, n_q)) != NOMAS_OK) return st;
+  if ((st = rows_map(&a.tmap_q, q, n_q, 128, heads)) != NOMAS_OK) return st;
+  a.heads = heads;
   const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)kHeadDim);
   a.scale_log2 = (float)(scale * 1.4426950408889634);
   a.n_spans = n_used;

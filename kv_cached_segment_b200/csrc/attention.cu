@@ -349,7 +349,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
   const int g1 = (int)((int64_t)total_tiles * (blockIdx.z + 1) / p.kv_splits);
   int n_kv = g1 - g0;  // K/V tiles this block streams
   if constexpr (kSparse) {
-    const int64_t row = (int64_t)blockIdx.x * kHeads + head;
+    const int64_t row = (int64_t)blockIdx.x * p.heads + head;
     list = p.tile_list + row * p.max_tiles;
     n_list = min(max(p.tile_count[row], 0), p.max_tiles);
     n_kv = 0;
@@ -517,7 +517,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
           const int64_t key = (int64_t)kt * kBN + r;
           const bool in_span = key < p.span_len[0];
           for (int which = 0; which < 2; ++which, ++t, ++u) {
-            const float scale = in_span ? __ldg(p.i8_scale[which] + key * kHeads + head) : 0.f;
+            const float scale = in_span ? __ldg(p.i8_scale[which] + key * p.heads + head) : 0.f;
             const int st = u & 1;
             const int slot = t % kStages;
             const bool got =
@@ -724,15 +724,16 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       lse_base = p.owner_lse[s];
       part = p.owner_slot;
     }
-    uint16_t *const o_out = o_base + part * p.n_q * kRowElems;
-    float *const lse_out = lse_base == nullptr ? nullptr : lse_base + part * kHeads * p.n_q;
+    const int64_t row_elems = (int64_t)p.heads * kHeadDim;
+    uint16_t *const o_out = o_base + part * p.n_q * row_elems;
+    float *const lse_out = lse_base == nullptr ? nullptr : lse_base + part * p.heads * p.n_q;
     bool have_o = ok && n_kv > 0;
     if (have_o) have_o = __all_sync(0xffffffffu, wait_phase(bar(kBarOFull + tile), 0, ctl));
     if (have_o) {
       tc_fence_after();
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       const float inv_l = 1.0f / l;
-      uint16_t *orow_g = o_out + row * kRowElems + head * kHeadDim;
+      uint16_t *orow_g = o_out + row * row_elems + head * kHeadDim;
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         uint32_t orow[32];
@@ -763,7 +764,7 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
       const uint32_t fill = empty ? 0u : 0x7FC07FC0u;  // bf16 0 or quiet NaN pairs
       const int64_t row = (int64_t)q_row0 + tile * kBM + quarter * 32 + lane;
       if (row < p.n_q) {
-        uint4 *dst = reinterpret_cast<uint4 *>(o_out + row * kRowElems + head * kHeadDim);
+        uint4 *dst = reinterpret_cast<uint4 *>(o_out + row * row_elems + head * kHeadDim);
 #pragma unroll
         for (int v = 0; v < 16; ++v) dst[v] = make_uint4(fill, fill, fill, fill);
         if (lse_out != nullptr) lse_out[(int64_t)head * p.n_q + row] = empty ? -INFINITY : NAN;
@@ -808,13 +809,13 @@ attention_kernel(const __grid_constant__ AttnArgs p) {
 }
 
 // Zero keys: O = 0, LSE = -inf.
-__global__ void attention_empty_kernel(uint16_t *o, float *lse, int64_t n_q) {
+__global__ void attention_empty_kernel(uint16_t *o, float *lse, int64_t n_q, int32_t heads) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t n_vec = n_q * kRowVecs;
+  const int64_t n_vec = n_q * heads * (kHeadDim * 2 / 16);
   for (int64_t v = i; v < n_vec; v += (int64_t)gridDim.x * blockDim.x)
     reinterpret_cast<uint4 *>(o)[v] = make_uint4(0, 0, 0, 0);
   if (lse != nullptr)
-    for (int64_t v = i; v < n_q * kHeads; v += (int64_t)gridDim.x * blockDim.x) lse[v] = -INFINITY;
+    for (int64_t v = i; v < n_q * heads; v += (int64_t)gridDim.x * blockDim.x) lse[v] = -INFINITY;
 }
 
 }  // namespace
@@ -855,7 +856,8 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   if (a.kv_splits < 1 || a.kv_splits > NOMAS_MAX_MERGE_PARTS ||
       (a.kv_splits > 1 && (a.tile_list != nullptr || a.lse == nullptr)))
     return cudaErrorInvalidValue;
-  dim3 grid((unsigned)q_blocks, kHeads, (unsigned)a.kv_splits);
+  if (a.heads < 1 || a.heads > kHeads) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)q_blocks, (unsigned)a.heads, (unsigned)a.kv_splits);
   if (a.i8) {
     if (a.tile_list != nullptr) return cudaErrorInvalidValue;
     if (state != 1) return cudaErrorInvalidKernelImage;
@@ -869,9 +871,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q, cudaStream_t stream) {
+cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q, int32_t heads,
+                                   cudaStream_t stream) {
   if (n_q <= 0) return cudaSuccess;
-  attention_empty_kernel<<<1184, 256, 0, stream>>>(o, lse, n_q);
+  attention_empty_kernel<<<1184, 256, 0, stream>>>(o, lse, n_q, heads);
   return cudaGetLastError();
 }
 

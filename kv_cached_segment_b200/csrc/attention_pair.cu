@@ -660,10 +660,11 @@ attention_pair_kernel(const __grid_constant__ AttnArgs p) {
       lse_base = p.owner_lse[so];
       part = p.owner_slot;
     }
-    uint16_t *const o_out = o_base + part * p.n_q * kRowElems;
-    float *const lse_out = lse_base == nullptr ? nullptr : lse_base + part * kHeads * p.n_q;
+    const int64_t row_elems = (int64_t)p.heads * kHeadDim;
+    uint16_t *const o_out = o_base + part * p.n_q * row_elems;
+    float *const lse_out = lse_base == nullptr ? nullptr : lse_base + part * p.heads * p.n_q;
     uint4 *const dst =
-        reinterpret_cast<uint4 *>(o_out + my_row * kRowElems + head * kHeadDim + 64 * h);
+        reinterpret_cast<uint4 *>(o_out + my_row * row_elems + head * kHeadDim + 64 * h);
     if (have_o) {
       tc_fence_after();
       const float inv_l = 1.0f / l_row;
@@ -741,7 +742,7 @@ cudaError_t launch_attention_pair(const AttnArgs &a, bool pair, cudaStream_t str
     if (e != cudaSuccess) return e;
     attr_set[dev].store(1, std::memory_order_release);
   }
-  if (!attention_pair_supported(a)) return cudaErrorInvalidValue;
+  if (!attention_pair_supported(a) || a.heads < 1 || a.heads > kHeads) return cudaErrorInvalidValue;
   if (a.kv_splits < 1 || a.kv_splits > NOMAS_MAX_MERGE_PARTS || (a.kv_splits > 1 && a.lse == nullptr))
     return cudaErrorInvalidValue;
   const int64_t units = ((int64_t)a.n_q + 2 * kRows - 1) / (2 * kRows);  // 256-row units
@@ -749,12 +750,12 @@ cudaError_t launch_attention_pair(const AttnArgs &a, bool pair, cudaStream_t str
   if (units > 0x3fffffff) return cudaErrorInvalidValue;
   if (!pair) {
     const int64_t blocks = ((int64_t)a.n_q + kRows - 1) / kRows;
-    dim3 grid((unsigned)blocks, kHeads, (unsigned)a.kv_splits);
+    dim3 grid((unsigned)blocks, (unsigned)a.heads, (unsigned)a.kv_splits);
     attention_pair_kernel<false><<<grid, kThreads, PCfg<false>::kSmemAlloc, stream>>>(a);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(2 * units), kHeads, (unsigned)a.kv_splits);
+  cfg.gridDim = dim3((unsigned)(2 * units), (unsigned)a.heads, (unsigned)a.kv_splits);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = PCfg<true>::kSmemAlloc;
   cfg.stream = stream;

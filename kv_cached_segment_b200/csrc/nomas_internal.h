@@ -79,6 +79,8 @@ struct AttnArgs {
   CUtensorMap tmap_v[kMaxSpans];
   int64_t span_len[kMaxSpans];
   int32_t n_spans;             // non-empty spans, packed to the front
+  int32_t heads;               // heads per row of Q, K, V, O (16; fewer for head-sharded
+                               // dense calls): rows are heads x 128 elements
   int32_t n_q;
   uint16_t *o;
   float *lse;                  // may be null
@@ -117,7 +119,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
 // K/V tensor maps with 128-row (one-tile) or 64-row (pair) boxes.
 bool attention_pair_supported(const AttnArgs &a);
 cudaError_t launch_attention_pair(const AttnArgs &a, bool pair, cudaStream_t stream);
-cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q,
+cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q, int32_t heads,
                                    cudaStream_t stream);
 
 // ---------------------------------------------------------------- merge ----

@@ -456,3 +456,23 @@ def test_attention_pipeline_choice_validation(lib):
                                         128, None, None, None)
     assert st == nm.NOMAS_ERR_CUDA, lib.nomas_last_error()
     assert lib.nomas_set_attention_pipeline(0) == nm.NOMAS_OK
+
+
+def test_attention_head_counts(lib):
+    q, o = FAKE, FAKE + 10 ** 9
+    spans = (nm._KVSpan * 1)(nm._KVSpan(FAKE + 2 * 10 ** 9, FAKE + 3 * 10 ** 9, 300))
+    for heads in (3, 6, 12, 32, 0):
+        assert lib.nomas_segment_attention(q, 100, spans, 1, o, None, 0.0, heads, 128, None,
+                                           None) == nm.NOMAS_ERR_UNSUPPORTED
+    for heads in (1, 2, 4, 8):
+        # dense bf16: accepted (without a GPU driver it stops at the tensor map)
+        assert lib.nomas_segment_attention(q, 100, spans, 1, o, None, 0.0, heads, 128, None,
+                                           None) == nm.NOMAS_ERR_CUDA
+        # sparse, key-split and INT8 calls keep 16 heads
+        lists, counts, err = FAKE + 7 * 10 ** 9, FAKE + 8 * 10 ** 9, FAKE + 9 * 10 ** 9
+        assert lib.nomas_segment_attention_sparse(q, 100, spans, 1, lists, counts, 3, o, None, 0.0,
+                                                  heads, 128, err, None) == nm.NOMAS_ERR_UNSUPPORTED
+        hist = nm._KVSpanI8(FAKE + 4 * 10 ** 9, FAKE + 5 * 10 ** 9, FAKE + 6 * 10 ** 9,
+                            FAKE + 6 * 10 ** 9 + 10 ** 6, 1000)
+        assert lib.nomas_segment_attention_i8(q, 100, ctypes.byref(hist), spans, 1, o, None, 0.0,
+                                              heads, 128, None, None, None) == nm.NOMAS_ERR_UNSUPPORTED

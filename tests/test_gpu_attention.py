@@ -25,7 +25,7 @@ def pipeline(request):
 def _attn(q, spans, scale=0.0, want_lse=True):
     qd = q.cuda()
     sd = [(k.cuda(), v.cuda()) for k, v in spans]
-    lse = torch.empty(16 * q.shape[0], dtype=torch.float32, device="cuda") if want_lse else None
+    lse = torch.empty(q.shape[1] * q.shape[0], dtype=torch.float32, device="cuda") if want_lse else None
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     o = nm.segment_attention(qd, sd, lse=lse, softmax_scale=scale, dev_err=err)
     torch.cuda.synchronize()
@@ -237,3 +237,34 @@ def test_attention_logit_spike_in_later_tile(col, spike):
     v = randn_bf16((n_k, 16, 128), 51)
     o = _check(q, [(k, v)], what=f"spike {spike} at column {col}")
     assert_close(f64(o), np.broadcast_to(f64(v[128 + col]), (64, 16, 128)), what="spike row")
+
+
+@pytest.mark.parametrize("heads", [1, 2, 4, 8])
+def test_attention_fewer_heads_matches_oracle_and_full_run(heads):
+    # Rows of 1, 2, 4 or 8 heads: the local heads of head-sharded attention.
+    # Each head is computed alone, so the result equals the 16-head run's
+    # heads bit for bit, and the oracle within the bar.
+    n_q, lens = 300, [200, 37, 129]
+    q = randn_bf16((n_q, 16, 128), 70 + heads)
+    spans = [(randn_bf16((n, 16, 128), 80 + i), randn_bf16((n, 16, 128), 90 + i))
+             for i, n in enumerate(lens)]
+    o16, l16 = _attn(q, spans)
+    h0 = 16 - heads  # the last heads of the row
+    qs = q[:, h0:].contiguous()
+    ss = [(k[:, h0:].contiguous(), v[:, h0:].contiguous()) for k, v in spans]
+    o, lse = _attn(qs, ss)
+    assert torch.equal(o, o16[:, h0:].contiguous())
+    assert torch.equal(lse.view(heads, n_q), l16.view(16, n_q)[h0:])
+    o_ref, l_ref = oracle.attention(f64(qs), [(f64(k), f64(v)) for k, v in ss])
+    assert_close(f64(o), o_ref, what=f"{heads} heads O")
+    assert_close(lse.view(heads, -1).cpu().numpy().astype(np.float64), l_ref, what=f"{heads} heads LSE")
+
+
+def test_head_sharded_single_rank_is_plain_attention():
+    q = randn_bf16((257, 16, 128), 5).cuda()
+    k, v = randn_bf16((300, 16, 128), 6).cuda(), randn_bf16((300, 16, 128), 7).cuda()
+    lse = torch.empty(16 * 257, dtype=torch.float32, device="cuda")
+    o = nm.head_sharded_segment_attention(q, [(k[:100], v[:100]), (k[100:], v[100:])], lse=lse)
+    o_ref, l_ref = _attn(q.cpu(), [(k.cpu(), v.cpu())])
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)

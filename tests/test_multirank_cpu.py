@@ -188,3 +188,69 @@ def test_local_key_spans_partition_in_order():
                 base = sum(lens[:s])
                 seen.extend(range(base + lo, base + hi))
         assert seen == list(range(sum(lens)))
+
+
+def _head_sharded_worker(rank, world, port, out):
+    # Head-sharded (Ulysses-style) attention: query and key rows spread over
+    # the ranks, one all-to-all to heads, attention over 16/world heads, one
+    # all-to-all back; the oracle stands in for the kernel.
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+
+    import kv_cached_segment_b200 as nm
+    import oracle
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(2)
+        lens = [70, 9, 40]
+        q = torch.randn((23, 16, 128), generator=g, dtype=torch.float64)
+        kv = [(torch.randn((n, 16, 128), generator=g, dtype=torch.float64),
+               torch.randn((n, 16, 128), generator=g, dtype=torch.float64)) for n in lens]
+        qa, qb = nm.shard_rows(23, rank, world, align=1)
+        spans = []
+        for k, v in kv:
+            a, b = nm.shard_rows(k.shape[0], rank, world, align=1)
+            if b > a:
+                spans.append((k[a:b], v[a:b]))
+        seen = {}
+
+        def attend(qq, sp, lse_out):
+            seen["heads"] = qq.shape[1]
+            seen["rows"] = qq.shape[0]
+            seen["keys"] = sum(a.shape[0] for a, _ in sp)
+            o, l = oracle.attention(qq.numpy(), [(a.numpy(), b.numpy()) for a, b in sp])
+            lse_out.copy_(torch.from_numpy(l).reshape(-1))
+            return torch.from_numpy(o)
+
+        lse = torch.empty(16 * (qb - qa), dtype=torch.float32)
+        o = nm.head_sharded_segment_attention(q[qa:qb], spans, attend=attend, lse=lse)
+        o_ref, l_ref = oracle.attention(q.numpy(), [(a.numpy(), b.numpy()) for a, b in kv])
+        out[rank] = (float(np.abs(o.numpy() - o_ref[qa:qb]).max()),
+                     float(np.abs(lse.view(16, -1).double().numpy() - l_ref[:, qa:qb]).max()),
+                     seen["heads"], seen["rows"], seen["keys"])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_attention_on_gloo_ranks():
+    for world in (2, 4):
+        ctx = mp.get_context("spawn")
+        mgr = ctx.Manager()
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_head_sharded_worker, args=(r, world, port, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=180)
+            assert p.exitcode == 0
+        for r in range(world):
+            err_o, err_l, heads, rows, keys = out[r]
+            assert err_o < 1e-9 and err_l < 1e-5, (world, r, err_o, err_l)
+            # every rank attends over all rows and all keys for 16/world heads
+            assert heads == 16 // world and rows == 23 and keys == 70 + 9 + 40
