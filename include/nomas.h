@@ -16,8 +16,9 @@
  *     16 x 128 bf16 is 4096 bytes.  Every tensor pointer must be 16-byte
  *     aligned.
  *   - Only heads = 16 and head_dim = 128 are implemented (and 1, 2, 4 or 8
- *     heads for nomas_segment_attention and nomas_segment_attention_ex on
- *     dense bf16 spans); other values return NOMAS_ERR_UNSUPPORTED.
+ *     heads for dense bf16 attention -- nomas_segment_attention, _ex, _split
+ *     and _split_noalloc -- and for nomas_attention_merge); other values
+ *     return NOMAS_ERR_UNSUPPORTED.
  *   - Every call is asynchronous on the caller's stream (`stream` is a
  *     cudaStream_t; NULL is the legacy default stream) and never synchronises.
  *     Argument errors are detected on the host before anything is launched and

@@ -463,7 +463,8 @@ def kvcache_select(src, frame_idx, window, dev_err=None, stream=None) -> None:
     del keep
 
 
-def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8) -> int:
+def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8,
+                   heads: int = HEADS) -> int:
     """Key splits for ``segment_attention(kv_splits="auto")``.
 
     Minimises a simple time model of the launch, in units of one CTA's time
@@ -472,7 +473,7 @@ def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8
     the S partial rows (read at ~5.5 TB/s, one tile taking ~1.5 us).  A
     split must leave at least 4 tiles per CTA and gain at least 2%."""
     tiles = sum((int(n) + 127) // 128 for n in span_lens)
-    ctas = (int(n_q) + 255) // 256 * HEADS
+    ctas = (int(n_q) + 255) // 256 * int(heads)
     if tiles == 0 or ctas == 0:
         return 1
     best, best_t = 1, None
@@ -481,7 +482,7 @@ def auto_kv_splits(n_q: int, span_lens, sm_count: int = 148, max_splits: int = 8
             break
         t = -(-ctas * s // sm_count) * (tiles / s + 3.0)
         if s > 1:
-            t += (s + 1) * n_q * (16 * 128 * 2 + 16 * 4) / 5.5e12 / 1.5e-6 + 3.0
+            t += (s + 1) * n_q * heads * (128 * 2 + 4) / 5.5e12 / 1.5e-6 + 3.0
         if best_t is None or t < 0.98 * best_t:
             best, best_t = s, t
     return best
@@ -520,10 +521,8 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         history, spans = spans[0]._c(), list(spans[1:])
         if kv_splits not in (1, "1"):
             raise ValueError("an INT8 history span takes kv_splits=1")
-    if heads != HEADS and kv_splits == "auto":
-        kv_splits = 1
-    if heads != HEADS and (history is not None or kv_splits not in (1, "1")):
-        raise ValueError("fewer than 16 heads: dense bf16 spans and kv_splits=1 only")
+    if heads != HEADS and history is not None:
+        raise ValueError("fewer than 16 heads: dense bf16 spans only")
     arr = (_KVSpan * max(1, len(spans)))()
     for i, (k, v) in enumerate(spans):
         nk = _rows(k, f"span {i} k", heads)
@@ -534,7 +533,7 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         raise TypeError("dev_err must be a CUDA int32 tensor")
     if kv_splits == "auto":
         sm = torch.cuda.get_device_properties(q.device).multi_processor_count
-        kv_splits = auto_kv_splits(n_q, [int(k.shape[0]) for k, _ in spans], sm)
+        kv_splits = auto_kv_splits(n_q, [int(k.shape[0]) for k, _ in spans], sm, heads=heads)
     kv_splits = int(kv_splits)
     if history is not None:
         opts = _AttnOpts(int(wait_limit_ns), int(testing_skip_kv_load), int(pipeline))
@@ -551,7 +550,7 @@ def segment_attention(q, spans, o=None, lse=None, softmax_scale: float = 0.0, de
         nbytes = lib.nomas_segment_attention_scratch_bytes(n_q, kv_splits)
         scratch = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
         _check(lib.nomas_segment_attention_split(_ptr(q), n_q, arr, len(spans), _ptr(o), _ptr(lse),
-                                                 float(softmax_scale), HEADS, HEAD_DIM, kv_splits,
+                                                 float(softmax_scale), heads, HEAD_DIM, kv_splits,
                                                  _ptr(scratch), nbytes, _ptr(dev_err),
                                                  _stream(stream)))
         # allocated on the current stream; when the kernels run on another

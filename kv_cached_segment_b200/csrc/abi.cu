@@ -565,8 +565,10 @@ nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, 
                                    int64_t n_q, void *o, float *lse, int32_t heads,
                                    int32_t head_dim, void *stream) {
   const ApiRange nvtx_range("nomas_attention_merge");
-  nomas_status st = check_shape(heads, head_dim);
-  if (st != NOMAS_OK) return st;
+  if (head_dim != kHeadDim || !(heads == 1 || heads == 2 || heads == 4 || heads == 8 ||
+                                heads == kHeads))
+    return fail(NOMAS_ERR_UNSUPPORTED, "heads=%d, head_dim=%d not implemented (1, 2, 4, 8 or 16 "
+                "heads of 128)", heads, head_dim);
   if (n_parts <= 0 || n_q < 0 || n_q > 0x7fff0000LL)
     return fail(NOMAS_ERR_INVALID_ARG, "need n_parts >= 1 and 0 <= n_q < 2^31");
   if (n_parts > NOMAS_MAX_MERGE_PARTS)
@@ -576,14 +578,15 @@ nomas_status nomas_attention_merge(const void *o_parts, const float *lse_parts, 
       !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return fail(NOMAS_ERR_INVALID_ARG, "merge pointers missing or misaligned");
-  const int64_t pb = (int64_t)n_parts * n_q * kRowBytes, lb = (int64_t)n_parts * n_q * kHeads * 4;
-  const int64_t ob = n_q * kRowBytes, olb = n_q * kHeads * 4;
+  const int64_t rb = (int64_t)heads * kHeadDim * 2, lr = (int64_t)heads * 4;
+  const int64_t pb = (int64_t)n_parts * n_q * rb, lb = (int64_t)n_parts * n_q * lr;
+  const int64_t ob = n_q * rb, olb = n_q * lr;
   if (overlap(o, ob, o_parts, pb) || overlap(o, ob, lse_parts, lb) ||
       (lse != nullptr && (overlap(lse, olb, o_parts, pb) || overlap(lse, olb, lse_parts, lb) ||
                           overlap(lse, olb, o, ob))))
     return fail(NOMAS_ERR_INVALID_ARG, "merge outputs overlap the inputs");
   const cudaError_t e = launch_merge(static_cast<const uint16_t *>(o_parts), lse_parts, n_parts,
-                                     n_q, static_cast<uint16_t *>(o), lse,
+                                     n_q, heads, static_cast<uint16_t *>(o), lse,
                                      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
@@ -742,15 +745,15 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                               int32_t kv_splits, void *scratch, int64_t scratch_bytes,
                               const OwnerRouting *routing, void *stream,
                               const nomas_kv_span_i8 *i8_span) {
-  // Heads per row: 16, or for a dense bf16 call without key splits or routed
-  // outputs 1, 2, 4 or 8 (the local heads of a head-sharded layout).
+  // Heads per row: 16, or for a dense bf16 call without routed outputs 1, 2,
+  // 4 or 8 (the local heads of a head-sharded layout).
   const bool few_heads_ok = (i8_span == nullptr || i8_span->len == 0) && tile_list == nullptr &&
-                            kv_splits == 1 && routing == nullptr;
+                            routing == nullptr;
   if (head_dim != kHeadDim ||
       !(heads == kHeads || (few_heads_ok && (heads == 1 || heads == 2 || heads == 4 || heads == 8))))
     return fail(NOMAS_ERR_UNSUPPORTED,
                 "heads=%d, head_dim=%d not implemented (16 heads of 128; 1, 2, 4 or 8 heads for "
-                "dense bf16 calls without key splits)", heads, head_dim);
+                "dense bf16 calls)", heads, head_dim);
   nomas_status st = NOMAS_OK;
   // Bytes of one row of Q, K, V or O, and of one query's LSE values.
   const int64_t row_bytes = (int64_t)heads * kHeadDim * 2, lse_row = (int64_t)heads * 4;
@@ -918,7 +921,7 @@ nomas_status attention_common(const void *q, int64_t n_q, const nomas_kv_span *s
                 "launch; refusing to run its register split", 128);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (kv_splits > 1) {
-    e = launch_merge(part_o, part_lse, kv_splits, n_q, static_cast<uint16_t *>(o), lse,
+    e = launch_merge(part_o, part_lse, kv_splits, n_q, heads, static_cast<uint16_t *>(o), lse,
                      static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "merge of key splits launch");
   }

@@ -10,11 +10,12 @@
 // reads the R shard LSEs of its (row, head) -- consecutive threads read
 // consecutive rows, so the reads coalesce -- and leaves the normalised
 // weights e^{LSE_r - LSE} in shared memory, and the merged LSE in global
-// memory.  Phase 2: the block walks its rows; for each, thread (head, chunk)
-// owns one 16-byte chunk (8 dims), reads the R partial chunks (the 256
-// threads cover one 4 KiB row, so every part's row is one coalesced read),
-// four parts in flight at a time, and accumulates in fp32.
-// Traffic per row: R x (4 KiB + 64 B) read + 4 KiB + 64 B written.
+// memory.  Phase 2: the block walks its rows; thread (head, chunk) owns one
+// 16-byte chunk (8 dims) of a row, reads the R partial chunks (256 threads
+// cover 4 KiB of rows, so every part's rows are one coalesced read), four
+// parts in flight at a time, and accumulates in fp32.  Rows hold H heads
+// (16, or fewer for head-sharded attention): 16 / H rows per pass.
+// Traffic per row: R x (H x 256 B + 4 H B) read + H x 256 B + 4 H B written.
 //
 // The same kernel serves two layouts of the partials: stacked in one buffer
 // (nomas_attention_merge, all rows, one output), or found through a table of
@@ -23,6 +24,8 @@
 // the merge in one kernel: each GPU reads the partial rows it owns from every
 // GPU and stores the merged rows into every GPU's output, with plain loads
 // and stores over NVLink.
+#include <type_traits>
+
 #include <cuda_bf16.h>
 
 #include "nomas_internal.h"
@@ -34,19 +37,22 @@ constexpr int kRows = 16;                  // query rows per block
 constexpr int kThreads = kRows * kHeads;   // phase 1: one (row, head) per thread
 constexpr int kWRow = kHeads + 1;          // padded [row][head] plane of one part
 constexpr int kWPlane = kRows * kWRow;
+constexpr int kChunks = kHeadDim * 2 / 16;  // 16-byte chunks per head
 
 // Where the R partial results live.  Stacked: one buffer, part r at a fixed
-// stride ([R][n_q][16][128] and [R][16][n_q]).  Table: R base pointers, any
-// of which may address another GPU's memory mapped into this process.
+// stride ([R][n_q][H][128] and [R][H][n_q]).  Table (16 heads): R base
+// pointers, any of which may address another GPU's memory mapped into this
+// process.
+template <int H>
 struct StackedParts {
   const uint16_t *o;
   const float *lse;
   int64_t n_q;
   __device__ __forceinline__ const uint4 *o_row(int r, int64_t row) const {
-    return reinterpret_cast<const uint4 *>(o) + ((int64_t)r * n_q + row) * kRowVecs;
+    return reinterpret_cast<const uint4 *>(o) + ((int64_t)r * n_q + row) * (H * kChunks);
   }
   __device__ __forceinline__ float lse_at(int r, int h, int64_t row) const {
-    return lse[((int64_t)r * kHeads + h) * n_q + row];
+    return lse[((int64_t)r * H + h) * n_q + row];
   }
 };
 struct TableParts {
@@ -54,7 +60,7 @@ struct TableParts {
   const float *lse[NOMAS_MAX_MERGE_PARTS];
   int64_t n_q;
   __device__ __forceinline__ const uint4 *o_row(int r, int64_t row) const {
-    return reinterpret_cast<const uint4 *>(o[r]) + row * kRowVecs;
+    return reinterpret_cast<const uint4 *>(o[r]) + row * (kHeads * kChunks);
   }
   __device__ __forceinline__ float lse_at(int r, int h, int64_t row) const {
     return lse[r][(int64_t)h * n_q + row];
@@ -68,13 +74,13 @@ struct Outputs {
   int32_t n;
 };
 
-template <class Parts>
+template <class Parts, int H>
 __global__ void __launch_bounds__(kThreads)
 merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
              int64_t row_end, const Outputs outs) {
   extern __shared__ float w_s[];  // [n_parts][kRows][kWRow]
   const int64_t row0 = row_begin + (int64_t)blockIdx.x * kRows;
-  {
+  if (threadIdx.x < kRows * H) {
     const int h = threadIdx.x >> 4, rr = threadIdx.x & 15;
     const int64_t row = row0 + rr;
     float *w = w_s + rr * kWRow + h;
@@ -103,8 +109,11 @@ merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
     }
   }
   __syncthreads();
-  const int h = threadIdx.x >> 4, c = threadIdx.x & 15;
-  for (int i = 0; i < kRows; ++i) {
+  // Phase 2: H x 16 chunks per row, 16 / H rows per pass, H passes.
+  const int chunk = threadIdx.x % (H * kChunks);
+  const int h = chunk / kChunks;
+  for (int pass = 0; pass < H; ++pass) {
+    const int i = pass * (kThreads / (H * kChunks)) + (int)threadIdx.x / (H * kChunks);
     const int64_t row = row0 + i;
     if (row >= row_end) break;
     const float *w = w_s + i * kWRow + h;
@@ -117,7 +126,7 @@ merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
         acc[2 * k + 1] = fmaf(wr, __uint_as_float(wd[k] & 0xffff0000u), acc[2 * k + 1]);
       }
     };
-    const int off = h * 16 + c;  // this thread's 16-byte chunk of the row
+    const int off = chunk;  // this thread's 16-byte chunk of the row
     int r = 0;
     for (; r + 4 <= n_parts; r += 4) {
       uint4 v[4];
@@ -135,14 +144,14 @@ merge_kernel(const Parts parts, int32_t n_parts, int64_t n_q, int64_t row_begin,
     }
     const uint4 packed = make_uint4(out[0], out[1], out[2], out[3]);
     for (int k = 0; k < outs.n; ++k)
-      reinterpret_cast<uint4 *>(outs.o[k] + row * kRowElems)[off] = packed;
+      reinterpret_cast<uint4 *>(outs.o[k] + row * (H * kHeadDim))[off] = packed;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_t n_parts,
-                         int64_t n_q, uint16_t *o, float *lse, cudaStream_t stream) {
+                         int64_t n_q, int32_t heads, uint16_t *o, float *lse, cudaStream_t stream) {
   if (n_q <= 0) return cudaSuccess;
   const int64_t blocks = (n_q + kRows - 1) / kRows;
   if (blocks > 0x7fffffff || n_parts > NOMAS_MAX_MERGE_PARTS) return cudaErrorInvalidValue;
@@ -151,8 +160,19 @@ cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_
   outs.o[0] = o;
   outs.lse[0] = lse;
   outs.n = 1;
-  merge_kernel<StackedParts><<<(unsigned)blocks, kThreads, smem, stream>>>(
-      StackedParts{o_parts, lse_parts, n_q}, n_parts, n_q, 0, n_q, outs);
+  auto go = [&](auto hc) {
+    constexpr int H = decltype(hc)::value;
+    merge_kernel<StackedParts<H>, H><<<(unsigned)blocks, kThreads, smem, stream>>>(
+        StackedParts<H>{o_parts, lse_parts, n_q}, n_parts, n_q, 0, n_q, outs);
+  };
+  switch (heads) {
+    case 1: go(std::integral_constant<int, 1>{}); break;
+    case 2: go(std::integral_constant<int, 2>{}); break;
+    case 4: go(std::integral_constant<int, 4>{}); break;
+    case 8: go(std::integral_constant<int, 8>{}); break;
+    case kHeads: go(std::integral_constant<int, kHeads>{}); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
@@ -178,7 +198,7 @@ cudaError_t launch_merge_peers(const uint16_t *const *o_parts, const float *cons
   }
   outs.n = n_outs;
   const size_t smem = (size_t)n_parts * kWPlane * sizeof(float);
-  merge_kernel<TableParts><<<(unsigned)blocks, kThreads, smem, stream>>>(
+  merge_kernel<TableParts, kHeads><<<(unsigned)blocks, kThreads, smem, stream>>>(
       parts, n_parts, n_q, row0, row0 + n_rows, outs);
   return cudaGetLastError();
 }

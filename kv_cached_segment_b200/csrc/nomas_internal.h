@@ -123,8 +123,9 @@ cudaError_t launch_attention_empty(uint16_t *o, float *lse, int64_t n_q, int32_t
                                    cudaStream_t stream);
 
 // ---------------------------------------------------------------- merge ----
+// Rows of `heads` heads (1, 2, 4, 8 or 16).
 cudaError_t launch_merge(const uint16_t *o_parts, const float *lse_parts, int32_t n_parts,
-                         int64_t n_q, uint16_t *o, float *lse, cudaStream_t stream);
+                         int64_t n_q, int32_t heads, uint16_t *o, float *lse, cudaStream_t stream);
 // Rows [row0, row0 + n_rows) of n_parts partials found through pointer
 // tables (host arrays), written to n_outs outputs.
 cudaError_t launch_merge_peers(const uint16_t *const *o_parts, const float *const *lse_parts,

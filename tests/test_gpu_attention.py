@@ -258,6 +258,16 @@ def test_attention_fewer_heads_matches_oracle_and_full_run(heads):
     o_ref, l_ref = oracle.attention(f64(qs), [(f64(k), f64(v)) for k, v in ss])
     assert_close(f64(o), o_ref, what=f"{heads} heads O")
     assert_close(lse.view(heads, -1).cpu().numpy().astype(np.float64), l_ref, what=f"{heads} heads LSE")
+    # key splits and their merge at the same head count: the 16-head split's heads
+    qd, sd = q.cuda(), [(k.cuda(), v.cuda()) for k, v in spans]
+    l16s = torch.empty(16 * n_q, dtype=torch.float32, device="cuda")
+    o16s = nm.segment_attention(qd, sd, lse=l16s, kv_splits=3)
+    ls = torch.empty(heads * n_q, dtype=torch.float32, device="cuda")
+    os_ = nm.segment_attention(qs.cuda(), [(k.cuda(), v.cuda()) for k, v in ss], lse=ls, kv_splits=3)
+    torch.cuda.synchronize()
+    assert torch.equal(os_, o16s[:, h0:].contiguous())
+    assert torch.equal(ls.view(heads, n_q), l16s.view(16, n_q)[h0:])
+    assert_close(f64(os_), o_ref, what=f"{heads} heads, 3 key splits O")
 
 
 def test_head_sharded_single_rank_is_plain_attention():
