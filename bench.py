@@ -65,6 +65,10 @@ def parse_args():
                         "GPUs: each rank holds one shard and the partials are all-gathered over "
                         "NCCL; on one GPU with more shards: every shard on that GPU (the per-GPU "
                         "work of key-sharded attention); 0 = one launch over all keys")
+    p.add_argument("--head-shards", type=int, default=0,
+                   help="on one GPU: attention in this many launches of 16/N heads each, with "
+                        "head-sliced copies of the rows (the per-GPU work of N-way head-sharded "
+                        "attention, all N shares on this GPU); 0 = one launch of 16 heads")
     p.add_argument("--kv-splits", default="1",
                    help="key splits of the attention launch (an integer, or 'auto': chosen from "
                         "the grid's wave count); 1 = one CTA per query block and head")
@@ -198,6 +202,7 @@ class LayerStep:
         self.select_kernel = "select_kernel"
         self.sparse = None
         self.shards = 0
+        self.head_shards = 0
         self.kv_splits = 1
 
     def use_key_shards(self, n_shards: int):
@@ -210,6 +215,36 @@ class LayerStep:
                                   device="cuda")
         self.part_lse = torch.empty((n_shards, 16, w.n_q), dtype=torch.float32, device="cuda")
         self.launches_per_step += n_shards  # n_shards attention launches + 1 merge, was 1
+
+    def use_head_shards(self, n_shards: int):
+        """Attention in `n_shards` launches of 16 / n_shards heads each: what
+        each GPU of head-sharded attention computes, all shares on this GPU.
+        Each share's history rows are resident in a head-sliced layout (as a
+        GPU of head-sharded attention holds its heads' cache); per step the
+        rotated Q and the text and segment K/V are copied into head-sliced
+        buffers and O back (the local data movement of the two all-to-alls),
+        and each launch picks its key splits (kv_splits="auto")."""
+        torch, w = self.torch, self.w
+        if 16 % n_shards:
+            raise SystemExit("--head-shards must divide 16")
+        self.head_shards = n_shards
+        hl = 16 // n_shards
+        sl = [slice(g * hl, (g + 1) * hl) for g in range(n_shards)]
+        self.head_slices = sl
+        if self.frames is not None:
+            raise SystemExit("--head-shards uses a workload without a frame window")
+        self.hist_g = [(self.cache.k[:w.n_cache, s].contiguous(), self.cache.v[:w.n_cache, s].contiguous())
+                       for s in sl]
+        self.q_g = [torch.empty((w.n_q, hl, 128), dtype=torch.bfloat16, device="cuda") for _ in sl]
+        self.o_g = [torch.empty_like(t) for t in self.q_g]
+        self.lse_g = [torch.empty(hl * w.n_q, dtype=torch.float32, device="cuda") for _ in sl]
+        self.ks_g = [torch.empty((w.n_text + w.n_seg, hl, 128), dtype=torch.bfloat16, device="cuda")
+                     for _ in sl]
+        self.vs_g = [torch.empty_like(t) for t in self.ks_g]
+        sm = torch.cuda.get_device_properties(0).multi_processor_count
+        splits = self.nm.auto_kv_splits(w.n_q, [w.n_cache, w.n_text + w.n_seg], sm, heads=hl)
+        # n_shards attention launches (was 1), and a merge each when keys are split
+        self.launches_per_step += n_shards - 1 + (n_shards if splits > 1 else 0)
 
     def _shard_spans(self, spans):
         lens = [int(k.shape[0]) for k, _ in spans]
@@ -273,6 +308,19 @@ class LayerStep:
         if self.sparse is not None:
             nm.segment_attention_sparse(self.q_rot, spans, *self.sparse, o=o, lse=self.lse,
                                         dev_err=self.err)
+        elif self.head_shards:
+            nt = w.n_text
+            for g, sl in enumerate(self.head_slices):
+                self.q_g[g].copy_(self.q_rot[:, sl])
+                self.ks_g[g][:nt].copy_(k[ns:, sl])
+                self.vs_g[g][:nt].copy_(v[ns:, sl])
+                self.ks_g[g][nt:].copy_(self.cache.k[w.n_cache:w.n_cache + ns, sl])
+                self.vs_g[g][nt:].copy_(self.cache.v[w.n_cache:w.n_cache + ns, sl])
+                nm.segment_attention(self.q_g[g], [self.hist_g[g], (self.ks_g[g], self.vs_g[g])],
+                                     o=self.o_g[g], lse=self.lse_g[g], dev_err=self.err,
+                                     kv_splits="auto")
+                o[:, sl].copy_(self.o_g[g])
+                self.lse.view(16, w.n_q)[sl].copy_(self.lse_g[g].view(-1, w.n_q))
         elif self.shards:
             for r, sub in enumerate(self._shard_spans(spans)):
                 nm.segment_attention(self.q_rot, sub, o=self.part_o[r],
@@ -703,6 +751,11 @@ def make_step(args, rank, world=1):
         if args.sparse > 0:
             raise SystemExit("--key-shards and --sparse are exclusive")
         step.use_key_shards(args.key_shards)
+    if args.head_shards > 0:
+        if world > 1 or args.sparse > 0 or args.key_shards > 0 or args.kv_splits != "1":
+            raise SystemExit("--head-shards runs on one GPU, dense, without key shards or "
+                             "--kv-splits (each launch picks its own)")
+        step.use_head_shards(args.head_shards)
     if args.kv_splits != "1":
         if not isinstance(step, LayerStep) or step.sparse is not None or step.shards:
             raise SystemExit("--kv-splits applies to the dense bf16 layer-step only")
@@ -734,6 +787,9 @@ def workload_text(args, step) -> str:
     if getattr(args, "key_shards", 0) > 0:
         extra += (f" (keys split into {args.key_shards} contiguous shards, partial results "
                   f"merged)")
+    if getattr(args, "head_shards", 0) > 0:
+        extra += (f" (heads split into {args.head_shards} launches of "
+                  f"{16 // args.head_shards} heads, rows copied to head-sliced buffers and back)")
     if args.sparse > 0:
         extra += (f" (block-sparse: text kept, {100 * args.sparse:.0f}% of video key tiles "
                   f"per 256-query block and head)")
@@ -1017,6 +1073,8 @@ def workload_config(args, step, world: int) -> dict:
     }
     if getattr(args, "key_shards", 0):
         cfg["key_shards"] = args.key_shards
+    if getattr(args, "head_shards", 0):
+        cfg["head_shards"] = args.head_shards
     return cfg
 
 
