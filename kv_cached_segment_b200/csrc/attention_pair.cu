@@ -38,6 +38,12 @@
 // Every wait is bounded (a globaltimer limit); on expiry the kernel records
 // NOMAS_DEVERR_WAIT_TIMEOUT, drains its own TMA loads and MMAs, sets the
 // block's rows of O and LSE to NaN, frees TMEM and returns.
+//
+// Both forms are selectable schedules, not the default: with one 128-row
+// tile per CTA the MMA lane's per-tile waits and commits are comparable to
+// the tile's 1,024 cycles of tensor work, and the pair's cross-CTA P
+// signalling at cluster scope is costly, so the two-tile kernel is faster on
+// every shape but the smallest.
 #include <atomic>
 
 #include <cuda_bf16.h>
